@@ -1,0 +1,195 @@
+"""CPU oracle for the ragged MoE grouped GEMM (fp64 over bf16 inputs).
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU
+baseline leg may import this package; the product library never does. It shares no code
+with the CUDA library. The arithmetic lives in ``gg_oracle.c`` (plain loops, OpenMP over
+rows); this module marshals numpy arrays into it.
+
+Definitions (see ``gg_oracle.c`` for the passages they follow):
+  forward  out[r,:] = A[r,:] @ W[e]            rows r of group e
+  dgrad    dX[r,:]  = dY[r,:] @ W[e]^T
+  wgrad    dW[e]    = A[group e]^T @ dY[group e]   (exact zeros for an empty group)
+  masked   out[e,r,:] = A[e,r,:] @ W[e]       r < clamp(masked_m[e], 0, mmax)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gg_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libgg_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (-O2 -fopenmp); returns the shared-library path."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+                           "-fno-fast-math", "-ffp-contract=off", _SRC, "-o", tmp, "-lm"])
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        i64, i32 = ctypes.c_int64, ctypes.c_int32
+        lib.gg_oracle_group_bounds.argtypes = [P, i32, i64, P, P]
+        lib.gg_oracle_group_bounds.restype = ctypes.c_int
+        for fn in (lib.gg_oracle_forward_rows, lib.gg_oracle_dgrad_rows):
+            fn.argtypes = [P, P, P, i32, i64, i64, i64, P, i64, P, P, ctypes.c_int]
+            fn.restype = None
+        lib.gg_oracle_wgrad_krows.argtypes = [P, P, P, i32, i64, i64, i64, P, i64, P,
+                                              ctypes.c_int]
+        lib.gg_oracle_wgrad_krows.restype = None
+        lib.gg_oracle_masked_forward_rows.argtypes = [P, P, P, i32, i64, i64, i64, P, i64,
+                                                      P, P, ctypes.c_int]
+        lib.gg_oracle_masked_forward_rows.restype = ctypes.c_int
+        lib.gg_oracle_round_bf16_array.argtypes = [P, i64, P]
+        lib.gg_oracle_round_bf16_array.restype = None
+        lib.gg_oracle_max_threads.restype = ctypes.c_int
+        _lib = lib
+        return lib
+
+
+def default_threads() -> int:
+    """Host cores available to this process."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def as_u16(x) -> np.ndarray:
+    """bf16 data as a C-contiguous uint16 numpy array (torch bf16 tensors or uint16)."""
+    if hasattr(x, "detach"):  # a torch tensor
+        import torch
+        t = x.detach()
+        if t.device.type != "cpu":
+            t = t.cpu()
+        return np.ascontiguousarray(t.contiguous().view(torch.int16).numpy().view(np.uint16))
+    a = np.asarray(x)
+    if a.dtype != np.uint16:
+        raise TypeError("bf16 data must be a torch.bfloat16 tensor or a uint16 array")
+    return np.ascontiguousarray(a)
+
+
+def _ptr(a: np.ndarray):
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def group_bounds(offs, rows_alloc: int):
+    """(starts, ends, bad): effective group bounds under the clamp rule."""
+    o = np.ascontiguousarray(np.asarray(offs, dtype=np.int32))
+    E = len(o)
+    s = np.zeros(E, np.int64)
+    e = np.zeros(E, np.int64)
+    bad = _load().gg_oracle_group_bounds(_ptr(o), E, rows_alloc, _ptr(s), _ptr(e))
+    return s, e, bool(bad)
+
+
+def _rows(rows, n):
+    if rows is None:
+        return np.arange(n, dtype=np.int64)
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    if r.size and (r.min() < 0 or r.max() >= n):
+        raise IndexError("row index out of range")
+    return r
+
+
+def forward(A, W, offs, rows=None, threads=None):
+    """fp64 forward on ``rows`` (default: all). Returns (out[nrows,N], group_of[nrows]);
+    rows in no group come back NaN with group -1."""
+    A, W = as_u16(A), as_u16(W)
+    o = np.ascontiguousarray(np.asarray(offs, dtype=np.int32))
+    rows_alloc, K = A.shape
+    E, K2, N = W.shape
+    assert K2 == K and len(o) == E
+    r = _rows(rows, rows_alloc)
+    out = np.empty((len(r), N), np.float64)
+    g = np.empty(len(r), np.int32)
+    _load().gg_oracle_forward_rows(_ptr(A), _ptr(W), _ptr(o), E, rows_alloc, K, N, _ptr(r),
+                                   len(r), _ptr(out), _ptr(g), threads or default_threads())
+    return out, g
+
+
+def dgrad(dY, W, offs, rows=None, threads=None):
+    """fp64 dgrad on ``rows``. Returns (dX[nrows,K], group_of[nrows])."""
+    dY, W = as_u16(dY), as_u16(W)
+    o = np.ascontiguousarray(np.asarray(offs, dtype=np.int32))
+    rows_alloc, N = dY.shape
+    E, K, N2 = W.shape
+    assert N2 == N and len(o) == E
+    r = _rows(rows, rows_alloc)
+    out = np.empty((len(r), K), np.float64)
+    g = np.empty(len(r), np.int32)
+    _load().gg_oracle_dgrad_rows(_ptr(dY), _ptr(W), _ptr(o), E, rows_alloc, K, N, _ptr(r),
+                                 len(r), _ptr(out), _ptr(g), threads or default_threads())
+    return out, g
+
+
+def wgrad(A, dY, offs, E=None, ks=None, threads=None):
+    """fp64 wgrad for the K-rows ``ks`` (default: all). Returns dW[E, len(ks), N]."""
+    A, dY = as_u16(A), as_u16(dY)
+    o = np.ascontiguousarray(np.asarray(offs, dtype=np.int32))
+    rows_alloc, K = A.shape
+    rows2, N = dY.shape
+    assert rows2 == rows_alloc
+    E = len(o) if E is None else E
+    assert len(o) == E
+    k = _rows(ks, K)
+    out = np.empty((E, len(k), N), np.float64)
+    _load().gg_oracle_wgrad_krows(_ptr(A), _ptr(dY), _ptr(o), E, rows_alloc, K, N, _ptr(k),
+                                  len(k), _ptr(out), threads or default_threads())
+    return out
+
+
+def masked_forward(A, W, masked_m, rows=None, threads=None):
+    """fp64 masked forward on flat rows e*mmax+r (default: all). Returns
+    (out[nrows,N], active[nrows], bad)."""
+    A, W = as_u16(A), as_u16(W)
+    m = np.ascontiguousarray(np.asarray(masked_m, dtype=np.int32))
+    E, mmax, K = A.shape
+    E2, K2, N = W.shape
+    assert E2 == E and K2 == K and len(m) == E
+    r = _rows(rows, E * mmax)
+    out = np.empty((len(r), N), np.float64)
+    act = np.empty(len(r), np.int32)
+    bad = _load().gg_oracle_masked_forward_rows(_ptr(A), _ptr(W), _ptr(m), E, mmax, K, N,
+                                                _ptr(r), len(r), _ptr(out), _ptr(act),
+                                                threads or default_threads())
+    return out, act.astype(bool), bool(bad)
+
+
+def round_bf16(x) -> np.ndarray:
+    """Round fp64 values to bf16 bit patterns (nearest, ties to even)."""
+    a = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+    out = np.empty(a.shape, np.uint16)
+    _load().gg_oracle_round_bf16_array(_ptr(a), a.size, _ptr(out))
+    return out
+
+
+def bf16_to_f64(u16) -> np.ndarray:
+    """Exact widening of bf16 bit patterns to fp64."""
+    a = np.asarray(u16, dtype=np.uint16).astype(np.uint32) << 16
+    return a.view(np.float32).astype(np.float64)
+
+
+def untouched_rows(offs, rows_alloc: int) -> np.ndarray:
+    """Rows of out/dX that no group covers (at and past the last effective end)."""
+    _, ends, _ = group_bounds(offs, rows_alloc)
+    last = int(ends[-1]) if len(ends) else 0
+    return np.arange(last, rows_alloc, dtype=np.int64)
