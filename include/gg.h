@@ -1,0 +1,147 @@
+/*
+ * gg.h -- ragged MoE grouped GEMM on NVIDIA B200 (sm_100a), C ABI.
+ *
+ * Operations (bf16 inputs, fp32 accumulation in tensor memory, bf16 outputs rounded to
+ * nearest even):
+ *
+ *   gg_forward         out[r,:] = A[r,:] . W[e]            for every row r of group e
+ *   gg_dgrad           dX[r,:]  = dY[r,:] . W[e]^T         for every row r of group e
+ *   gg_wgrad           dW[e]    = A[rows of e]^T . dY[rows of e]   (overwrite)
+ *   gg_masked_forward  out[e,r,:] = A[e,r,:] . W[e]        for r < masked_m[e]
+ *
+ * Groups. offs[E] holds cumulative END offsets with no leading zero: group e covers rows
+ * [offs[e-1], offs[e]) with offs[-1] = 0. This is the contract of torch._grouped_mm(x, w,
+ * offs) in PyTorch issue 152668 ("Easy repro scenario": 4 experts, offsets (8,16,32,40)
+ * over 48 rows, and the empty-expert variant (8,8,32,40)). A group may be empty and may have
+ * any size; no alignment is asked of the sizes (TransformerEngine PR 3224 names an
+ * alignment contract on m_splits that this library does not have).
+ *
+ * Offsets and masked_m are read only on the device ("expert counts remain on the GPU",
+ * TransformerEngine PR 3542, "Changes"). No call synchronises with the host, allocates
+ * memory, pads A or clears an output (TileOPs issue 1566, "Summary": the per-call zero
+ * fill and pad cost ~2.8 ms on a ~20 ms GEMM). Every call is ordered on the caller's
+ * stream and may be captured in a CUDA graph; the offsets may change between replays.
+ *
+ * Memory. All pointers are device pointers owned by the caller; bf16 arrays are row major
+ * (last index contiguous) and 16-byte aligned. W is one packed [E,K,N] buffer (the single
+ * grouped weight of TransformerEngine PR 3224). K and N must be multiples of 8.
+ *
+ * Untouched regions ("caller-owned output buffers and unused capacity are preserved",
+ * TransformerEngine PR 3542, "Changes"):
+ *   - out/dX rows at or past the last (effective) offset are never written, and A/dY rows
+ *     there are never read into any result;
+ *   - masked rows r >= masked_m[e] of out are never written; A rows there never reach a
+ *     result (sglang PR 32385, "Fix": masked_m excludes them from the GEMM);
+ *   - dW is always written in full; the dW of an empty expert is +0.0 everywhere.
+ *
+ * Errors. Problems visible on the host return a gg_status at once and launch nothing.
+ * Problems in device-resident data are never fatal: the kernel ORs a GG_DEV_* bit into
+ * *dev_status (when dev_status is not NULL), treats the offending group as described
+ * below, and still computes every valid group. No call traps, asserts or hangs: every wait
+ * inside a kernel is bounded by a watchdog, after which the kernel sets GG_DEV_TIMEOUT,
+ * drains its own copies in flight, frees its tensor memory and returns.
+ */
+#ifndef GG_H_
+#define GG_H_
+
+#include <stdint.h>
+#include <cuda_runtime.h>
+
+#if defined(__GNUC__)
+#define GG_API __attribute__((visibility("default")))
+#else
+#define GG_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GG_OK = 0,
+  GG_ERR_INVALID_ARG = 1,  /* null pointer, negative or zero size, E < 1, ...          */
+  GG_ERR_UNSUPPORTED = 2,  /* K or N not a multiple of 8, misaligned pointer, E too large,
+                              rows >= 2^31, or a device that is not sm_100                */
+  GG_ERR_CUDA = 3          /* a CUDA runtime/driver call failed (launch, attribute, ...) */
+} gg_status;
+
+/* Bits OR-ed into *dev_status by the kernels. */
+#define GG_DEV_BAD_OFFSETS  0x1u  /* an offset was negative, decreasing or > rows_alloc; the
+                                     effective ends t'_e = clamp(offs[e], t'_{e-1},
+                                     rows_alloc) (t'_{-1}=0) were used instead            */
+#define GG_DEV_BAD_MASKED_M 0x2u  /* a masked_m was < 0 or > mmax; it was clamped         */
+#define GG_DEV_TIMEOUT      0x4u  /* a pipeline wait exceeded the watchdog; results of this
+                                     call are incomplete                                  */
+#define GG_DEV_ERROR_MASK   0xFFu
+#define GG_DEV_LAUNCHED     0x100u /* informational: the sm_100a kernel ran to its end     */
+
+/* Largest expert count a call accepts. */
+#define GG_MAX_EXPERTS 1024
+
+/*
+ * Forward: out[r, n] = sum_k A[r, k] * W[e, k, n] for every row r of group e.
+ *   A    bf16 [rows_alloc, K]      read only for rows inside a group
+ *   W    bf16 [E, K, N]
+ *   offs int32 [E], device         cumulative end offsets
+ *   out  bf16 [rows_alloc, N]      rows inside a group overwritten; other rows untouched
+ *   dev_status int32, device, may be NULL
+ * Passage: PyTorch issue 152668, "Easy repro scenario" (o = torch._grouped_mm(x, w, offs)).
+ */
+GG_API gg_status gg_forward(const void* A, const void* W, const int32_t* offs, void* out,
+                     int64_t rows_alloc, int64_t K, int64_t N, int32_t E,
+                     int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * Dgrad: dX[r, k] = sum_n dY[r, n] * W[e, k, n] for every row r of group e.
+ *   dY bf16 [rows_alloc, N]; W bf16 [E, K, N]; dX bf16 [rows_alloc, K] (rows outside every
+ *   group untouched).
+ * Passage: PyTorch issue 152668 (o.backward: the grad of x over the same offsets);
+ * TransformerEngine PR 3542, "Changes" (forward, dgrad and wgrad through one grouped GEMM).
+ */
+GG_API gg_status gg_dgrad(const void* dY, const void* W, const int32_t* offs, void* dX,
+                   int64_t rows_alloc, int64_t K, int64_t N, int32_t E,
+                   int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * Wgrad: dW[e, k, n] = sum over rows r of group e of A[r, k] * dY[r, n].
+ *   A bf16 [rows_alloc, K]; dY bf16 [rows_alloc, N]; dW bf16 [E, K, N], written in full
+ *   (overwrite, not accumulate); an empty group yields +0.0.
+ * Passage: TransformerEngine PR 3542, "Changes" ("overwrite wgrad"); PyTorch issue 152668
+ * (the backward that must not hang on an empty expert).
+ */
+GG_API gg_status gg_wgrad(const void* A, const void* dY, const int32_t* offs, void* dW,
+                   int64_t rows_alloc, int64_t K, int64_t N, int32_t E,
+                   int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * Masked forward: out[e, r, n] = sum_k A[e, r, k] * W[e, k, n] for r < masked_m[e].
+ *   A bf16 [E, mmax, K]; W bf16 [E, K, N]; masked_m int32 [E], device;
+ *   out bf16 [E, mmax, N]: rows r >= masked_m[e] untouched.
+ * Passage: sglang PR 32385, "Evidence" and "Fix" (the masked grouped GEMM
+ * m_grouped_gemm_nt_masked(a, b, d, masked_m, expected_m); its expected-m hint has no
+ * counterpart here).
+ */
+GG_API gg_status gg_masked_forward(const void* A, const void* W, const int32_t* masked_m,
+                            void* out, int64_t mmax, int64_t K, int64_t N, int32_t E,
+                            int32_t* dev_status, cudaStream_t stream);
+
+/* A static, human-readable name for a status. */
+GG_API const char* gg_status_string(gg_status s);
+
+/* Watchdog bound of every in-kernel wait, in nanoseconds, for later calls from any
+   thread (default 4e9). Returns the previous value. 0 restores the default. */
+GG_API uint64_t gg_set_watchdog_ns(uint64_t ns);
+
+/* Test hook: when enable != 0, later calls make CTA 0's load warp skip its first stage,
+   so that the pipeline's first wait runs into the watchdog and the call reports
+   GG_DEV_TIMEOUT. No GPU fault is involved. Returns the previous setting. */
+GG_API int gg_testing_skip_first_load(int enable);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+GG_API int gg_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GG_H_ */

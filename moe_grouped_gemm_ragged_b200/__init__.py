@@ -1,0 +1,215 @@
+"""Ragged MoE grouped GEMM for B200 (sm_100a): a thin Python binding over ``libgg.so``.
+
+Every function here only checks and marshals arguments (device pointers, sizes, the current
+CUDA stream) into the C ABI declared in ``include/gg.h``; all arithmetic runs in the
+library's sm_100a kernels. There is no fallback: if the library is missing or cannot load,
+the import of the kernels fails with an error.
+
+Groups are cumulative END offsets (int32, on the device, no leading zero): group e covers
+rows [offs[e-1], offs[e]) with offs[-1] = 0, as in ``torch._grouped_mm(x, w, offs)``
+(PyTorch issue 152668, "Easy repro scenario").
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgg.so")
+
+GG_OK, GG_ERR_INVALID_ARG, GG_ERR_UNSUPPORTED, GG_ERR_CUDA = 0, 1, 2, 3
+DEV_BAD_OFFSETS = 0x1
+DEV_BAD_MASKED_M = 0x2
+DEV_TIMEOUT = 0x4
+DEV_ERROR_MASK = 0xFF
+DEV_LAUNCHED = 0x100
+MAX_EXPERTS = 1024
+
+_lib = None
+
+
+class GGError(RuntimeError):
+    """A non-OK status returned by the C ABI."""
+
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)}")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (``libgg.so``). Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m moe_grouped_gemm_ragged_b200._build`"
+            " (there is no non-CUDA implementation)")
+    L = ctypes.CDLL(LIB_PATH)
+    P, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+    sig = [P, P, P, P, i64, i64, i64, i32, P, P]
+    for name in ("gg_forward", "gg_dgrad", "gg_wgrad", "gg_masked_forward"):
+        fn = getattr(L, name)
+        fn.argtypes = sig
+        fn.restype = ctypes.c_int
+    L.gg_status_string.argtypes = [ctypes.c_int]
+    L.gg_status_string.restype = ctypes.c_char_p
+    L.gg_set_watchdog_ns.argtypes = [ctypes.c_uint64]
+    L.gg_set_watchdog_ns.restype = ctypes.c_uint64
+    L.gg_testing_skip_first_load.argtypes = [ctypes.c_int]
+    L.gg_testing_skip_first_load.restype = ctypes.c_int
+    L.gg_version.restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def status_string(code: int) -> str:
+    return lib().gg_status_string(int(code)).decode()
+
+
+def version() -> int:
+    return lib().gg_version()
+
+
+def set_watchdog_ns(ns: int) -> int:
+    """Bound of every in-kernel wait (ns) for later calls; returns the previous value."""
+    return int(lib().gg_set_watchdog_ns(int(ns)))
+
+
+def testing_skip_first_load(enable: bool) -> bool:
+    """Test hook: make later calls' first load go missing so the watchdog fires."""
+    return bool(lib().gg_testing_skip_first_load(1 if enable else 0))
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(t: torch.Tensor, name: str, dtype, ndim: int):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _status_ptr(status: Optional[torch.Tensor]):
+    if status is None:
+        return None
+    _check(status, "status", torch.int32, 1)
+    return status.data_ptr()
+
+
+def _raise(rc: int, where: str):
+    if rc != GG_OK:
+        raise GGError(rc, where)
+
+
+def forward(A: torch.Tensor, W: torch.Tensor, offs: torch.Tensor, out: torch.Tensor, *,
+            status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """out[r,:] = A[r,:] @ W[e] for every row r of group e; other rows of ``out`` untouched.
+
+    A bf16 [rows, K], W bf16 [E, K, N], offs int32 [E] (device), out bf16 [rows, N]."""
+    _check(A, "A", torch.bfloat16, 2)
+    _check(W, "W", torch.bfloat16, 3)
+    _check(offs, "offs", torch.int32, 1)
+    _check(out, "out", torch.bfloat16, 2)
+    rows, K = A.shape
+    E, K2, N = W.shape
+    if K2 != K or offs.numel() != E or tuple(out.shape) != (rows, N):
+        raise ValueError("shape mismatch: A[rows,K], W[E,K,N], offs[E], out[rows,N]")
+    rc = lib().gg_forward(_ptr(A), _ptr(W), _ptr(offs), _ptr(out), rows, K, N, E,
+                          _status_ptr(status), _stream_handle(stream))
+    _raise(rc, "gg_forward")
+    return out
+
+
+def dgrad(dY: torch.Tensor, W: torch.Tensor, offs: torch.Tensor, dX: torch.Tensor, *,
+          status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """dX[r,:] = dY[r,:] @ W[e]^T for every row r of group e; other rows untouched.
+
+    dY bf16 [rows, N], W bf16 [E, K, N], offs int32 [E], dX bf16 [rows, K]."""
+    _check(dY, "dY", torch.bfloat16, 2)
+    _check(W, "W", torch.bfloat16, 3)
+    _check(offs, "offs", torch.int32, 1)
+    _check(dX, "dX", torch.bfloat16, 2)
+    rows, N = dY.shape
+    E, K, N2 = W.shape
+    if N2 != N or offs.numel() != E or tuple(dX.shape) != (rows, K):
+        raise ValueError("shape mismatch: dY[rows,N], W[E,K,N], offs[E], dX[rows,K]")
+    rc = lib().gg_dgrad(_ptr(dY), _ptr(W), _ptr(offs), _ptr(dX), rows, K, N, E,
+                        _status_ptr(status), _stream_handle(stream))
+    _raise(rc, "gg_dgrad")
+    return dX
+
+
+def wgrad(A: torch.Tensor, dY: torch.Tensor, offs: torch.Tensor, dW: torch.Tensor, *,
+          status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """dW[e] = A[rows of e]^T @ dY[rows of e], all of dW overwritten (zeros if e is empty).
+
+    A bf16 [rows, K], dY bf16 [rows, N], offs int32 [E], dW bf16 [E, K, N]."""
+    _check(A, "A", torch.bfloat16, 2)
+    _check(dY, "dY", torch.bfloat16, 2)
+    _check(offs, "offs", torch.int32, 1)
+    _check(dW, "dW", torch.bfloat16, 3)
+    rows, K = A.shape
+    rows2, N = dY.shape
+    E = offs.numel()
+    if rows2 != rows or tuple(dW.shape) != (E, K, N):
+        raise ValueError("shape mismatch: A[rows,K], dY[rows,N], offs[E], dW[E,K,N]")
+    rc = lib().gg_wgrad(_ptr(A), _ptr(dY), _ptr(offs), _ptr(dW), rows, K, N, E,
+                        _status_ptr(status), _stream_handle(stream))
+    _raise(rc, "gg_wgrad")
+    return dW
+
+
+def masked_forward(A: torch.Tensor, W: torch.Tensor, masked_m: torch.Tensor,
+                   out: torch.Tensor, *, status: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    """out[e,r,:] = A[e,r,:] @ W[e] for r < masked_m[e]; other rows of ``out`` untouched.
+
+    A bf16 [E, mmax, K], W bf16 [E, K, N], masked_m int32 [E], out bf16 [E, mmax, N]."""
+    _check(A, "A", torch.bfloat16, 3)
+    _check(W, "W", torch.bfloat16, 3)
+    _check(masked_m, "masked_m", torch.int32, 1)
+    _check(out, "out", torch.bfloat16, 3)
+    E, mmax, K = A.shape
+    E2, K2, N = W.shape
+    if E2 != E or K2 != K or masked_m.numel() != E or tuple(out.shape) != (E, mmax, N):
+        raise ValueError("shape mismatch: A[E,mmax,K], W[E,K,N], masked_m[E], out[E,mmax,N]")
+    rc = lib().gg_masked_forward(_ptr(A), _ptr(W), _ptr(masked_m), _ptr(out), mmax, K, N, E,
+                                 _status_ptr(status), _stream_handle(stream))
+    _raise(rc, "gg_masked_forward")
+    return out
+
+
+def grouped_mm(A: torch.Tensor, W: torch.Tensor, offs: torch.Tensor,
+               out: Optional[torch.Tensor] = None, **kw) -> torch.Tensor:
+    """Forward with an optional caller-owned ``out`` (allocated uninitialised when None)."""
+    if out is None:
+        out = torch.empty((A.shape[0], W.shape[2]), dtype=A.dtype, device=A.device)
+    return forward(A, W, offs, out, **kw)
+
+
+__all__ = [
+    "forward", "dgrad", "wgrad", "masked_forward", "grouped_mm", "status_string", "version",
+    "set_watchdog_ns", "testing_skip_first_load", "lib", "GGError", "LIB_PATH",
+    "DEV_BAD_OFFSETS", "DEV_BAD_MASKED_M", "DEV_TIMEOUT", "DEV_ERROR_MASK", "DEV_LAUNCHED",
+    "MAX_EXPERTS",
+]

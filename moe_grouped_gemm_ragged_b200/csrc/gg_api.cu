@@ -1,0 +1,289 @@
+// C-ABI entry points of the ragged grouped GEMM: argument checks, TMA tensor-map encoding
+// and the persistent launch. No entry point reads the offsets on the host, allocates,
+// synchronises or clears memory; everything is ordered on the caller's stream.
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "gg.h"
+#include "gg_kernel.cuh"
+
+namespace {
+
+using gg::Mode;
+
+constexpr int kMaxDevices = 64;
+constexpr uint64_t kDefaultWatchdogNs = 4000000000ull;
+
+std::atomic<uint64_t> g_watchdog_ns{kDefaultWatchdogNs};
+std::atomic<int> g_skip_first_load{0};
+
+static_assert(gg::DEV_BAD_OFFSETS == GG_DEV_BAD_OFFSETS, "status bit mismatch");
+static_assert(gg::DEV_BAD_MASKED_M == GG_DEV_BAD_MASKED_M, "status bit mismatch");
+static_assert(gg::DEV_TIMEOUT == GG_DEV_TIMEOUT, "status bit mismatch");
+static_assert(gg::DEV_LAUNCHED == GG_DEV_LAUNCHED, "status bit mismatch");
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+struct DeviceInfo {
+  int sms = 0;
+  bool sm100 = false;
+  bool ready = false;
+};
+
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+gg_status device_info(DeviceInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GG_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return GG_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return GG_ERR_CUDA;
+    d.sms = sms;
+    d.sm100 = (major == 10 && minor == 0);
+    d.ready = true;
+  }
+  *out = d;
+  return GG_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Tiled bf16 tensor map with 128-byte swizzle; out-of-range elements read as zero.
+bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+              const uint64_t* strides_bytes, const uint32_t* box) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t gdim[3];
+  cuuint64_t gstr[2];
+  cuuint32_t bdim[3];
+  cuuint32_t estr[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    gdim[i] = dims[i];
+    bdim[i] = box[i];
+  }
+  for (int i = 0; i + 1 < rank; ++i) gstr[i] = strides_bytes[i];
+  std::memset(m, 0, sizeof(*m));
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
+                  gdim, gstr, bdim, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// 2-D map over a row-major [rows, cols] bf16 matrix.
+bool map_2d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_cols,
+            uint32_t box_rows) {
+  const uint64_t dims[2] = {(uint64_t)cols, (uint64_t)(rows > 0 ? rows : 1)};
+  const uint64_t str[1] = {(uint64_t)cols * 2u};
+  const uint32_t box[2] = {box_cols, box_rows};
+  return make_map(m, base, 2, dims, str, box);
+}
+
+// 3-D map over the packed weights W[E, K, N] (dims innermost first: N, K, E).
+bool map_w(CUtensorMap* m, const void* W, int64_t E, int64_t K, int64_t N, uint32_t box_n,
+           uint32_t box_k) {
+  const uint64_t dims[3] = {(uint64_t)N, (uint64_t)K, (uint64_t)E};
+  const uint64_t str[2] = {(uint64_t)N * 2u, (uint64_t)K * (uint64_t)N * 2u};
+  const uint32_t box[3] = {box_n, box_k, 1};
+  return make_map(m, W, 3, dims, str, box);
+}
+
+template <Mode MODE, int BN, int STAGES>
+gg_status launch(const CUtensorMap& a, const CUtensorMap& b, const gg::Params& p,
+                 int64_t tiles_upper, const DeviceInfo& di, cudaStream_t stream) {
+  auto kern = gg::grouped_gemm_kernel<MODE, BN, STAGES>;
+  const size_t smem = gg::Layout<BN, STAGES>::bytes(p.E);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GG_ERR_CUDA;
+  static bool attr_done[kMaxDevices] = {};
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (!attr_done[dev]) {
+      const int max_smem = (int)gg::Layout<BN, STAGES>::bytes(GG_MAX_EXPERTS);
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) !=
+          cudaSuccess)
+        return GG_ERR_CUDA;
+      attr_done[dev] = true;
+    }
+  }
+  int64_t grid = tiles_upper < di.sms ? tiles_upper : di.sms;
+  if (grid < 1) grid = 1;
+  kern<<<(unsigned)grid, gg::NUM_THREADS, smem, stream>>>(a, b, p);
+  return cudaGetLastError() == cudaSuccess ? GG_OK : GG_ERR_CUDA;
+}
+
+gg::Params base_params(const int32_t* groups, void* out, int32_t* status, int64_t rows_alloc,
+                       int32_t E) {
+  gg::Params p;
+  std::memset(&p, 0, sizeof(p));
+  p.groups = groups;
+  p.out = reinterpret_cast<__nv_bfloat16*>(out);
+  p.status = status;
+  p.rows_alloc = rows_alloc;
+  p.E = E;
+  p.watchdog_ns = g_watchdog_ns.load();
+  p.debug_flags = g_skip_first_load.load() ? 1 : 0;
+  return p;
+}
+
+gg_status check_common(int64_t rows_alloc, int64_t K, int64_t N, int32_t E,
+                       const int32_t* groups, const int32_t* dev_status, DeviceInfo* di) {
+  if (E < 1 || K < 1 || N < 1 || rows_alloc < 0 || groups == nullptr) return GG_ERR_INVALID_ARG;
+  if (E > GG_MAX_EXPERTS) return GG_ERR_UNSUPPORTED;
+  if ((K % 8) != 0 || (N % 8) != 0) return GG_ERR_UNSUPPORTED;
+  if (rows_alloc >= (int64_t(1) << 31) || K >= (int64_t(1) << 31) || N >= (int64_t(1) << 31))
+    return GG_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(groups) & 3u) != 0) return GG_ERR_UNSUPPORTED;
+  if (dev_status != nullptr && (reinterpret_cast<uintptr_t>(dev_status) & 3u) != 0)
+    return GG_ERR_UNSUPPORTED;
+  gg_status s = device_info(di);
+  if (s != GG_OK) return s;
+  if (!di->sm100) return GG_ERR_UNSUPPORTED;
+  return GG_OK;
+}
+
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+constexpr int kBN = 256;
+constexpr int kStages = 4;
+
+}  // namespace
+
+extern "C" {
+
+gg_status gg_forward(const void* A, const void* W, const int32_t* offs, void* out,
+                     int64_t rows_alloc, int64_t K, int64_t N, int32_t E, int32_t* dev_status,
+                     cudaStream_t stream) {
+  DeviceInfo di;
+  gg_status s = check_common(rows_alloc, K, N, E, offs, dev_status, &di);
+  if (s != GG_OK) return s;
+  if (W == nullptr) return GG_ERR_INVALID_ARG;
+  if (rows_alloc == 0) return GG_OK;  // no row can belong to a group
+  if (A == nullptr || out == nullptr) return GG_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(W) || !aligned16(out)) return GG_ERR_UNSUPPORTED;
+  CUtensorMap ma, mb;
+  if (!map_2d(&ma, A, rows_alloc, K, 64, gg::BM) || !map_w(&mb, W, E, K, N, 64, 64))
+    return GG_ERR_CUDA;
+  gg::Params p = base_params(offs, out, dev_status, rows_alloc, E);
+  p.red_len = (int32_t)K;
+  p.out_cols = (int32_t)N;
+  const int64_t tiles = (cdiv(rows_alloc, gg::BM) + E) * cdiv(N, kBN);
+  return launch<Mode::Forward, kBN, kStages>(ma, mb, p, tiles, di, stream);
+}
+
+gg_status gg_dgrad(const void* dY, const void* W, const int32_t* offs, void* dX,
+                   int64_t rows_alloc, int64_t K, int64_t N, int32_t E, int32_t* dev_status,
+                   cudaStream_t stream) {
+  DeviceInfo di;
+  gg_status s = check_common(rows_alloc, K, N, E, offs, dev_status, &di);
+  if (s != GG_OK) return s;
+  if (W == nullptr) return GG_ERR_INVALID_ARG;
+  if (rows_alloc == 0) return GG_OK;
+  if (dY == nullptr || dX == nullptr) return GG_ERR_INVALID_ARG;
+  if (!aligned16(dY) || !aligned16(W) || !aligned16(dX)) return GG_ERR_UNSUPPORTED;
+  CUtensorMap ma, mb;
+  if (!map_2d(&ma, dY, rows_alloc, N, 64, gg::BM) || !map_w(&mb, W, E, K, N, 64, kBN))
+    return GG_ERR_CUDA;
+  gg::Params p = base_params(offs, dX, dev_status, rows_alloc, E);
+  p.red_len = (int32_t)N;
+  p.out_cols = (int32_t)K;
+  const int64_t tiles = (cdiv(rows_alloc, gg::BM) + E) * cdiv(K, kBN);
+  return launch<Mode::Dgrad, kBN, kStages>(ma, mb, p, tiles, di, stream);
+}
+
+gg_status gg_wgrad(const void* A, const void* dY, const int32_t* offs, void* dW,
+                   int64_t rows_alloc, int64_t K, int64_t N, int32_t E, int32_t* dev_status,
+                   cudaStream_t stream) {
+  DeviceInfo di;
+  gg_status s = check_common(rows_alloc, K, N, E, offs, dev_status, &di);
+  if (s != GG_OK) return s;
+  if (dW == nullptr) return GG_ERR_INVALID_ARG;
+  if (!aligned16(dW)) return GG_ERR_UNSUPPORTED;
+  if (rows_alloc > 0) {
+    if (A == nullptr || dY == nullptr) return GG_ERR_INVALID_ARG;
+    if (!aligned16(A) || !aligned16(dY)) return GG_ERR_UNSUPPORTED;
+  } else {
+    // every group is empty: the maps are never used; dW only gets zeros
+    A = dW;
+    dY = dW;
+  }
+  CUtensorMap ma, mb;
+  if (!map_2d(&ma, A, rows_alloc, K, 64, 64) || !map_2d(&mb, dY, rows_alloc, N, 64, 64))
+    return GG_ERR_CUDA;
+  gg::Params p = base_params(offs, dW, dev_status, rows_alloc, E);
+  p.out_cols = (int32_t)N;
+  p.wg_K = (int32_t)K;
+  const int64_t tiles = (int64_t)E * cdiv(K, gg::BM) * cdiv(N, kBN);
+  return launch<Mode::Wgrad, kBN, kStages>(ma, mb, p, tiles, di, stream);
+}
+
+gg_status gg_masked_forward(const void* A, const void* W, const int32_t* masked_m, void* out,
+                            int64_t mmax, int64_t K, int64_t N, int32_t E, int32_t* dev_status,
+                            cudaStream_t stream) {
+  DeviceInfo di;
+  if (mmax < 0) return GG_ERR_INVALID_ARG;
+  if ((int64_t)E * mmax >= (int64_t(1) << 31)) return GG_ERR_UNSUPPORTED;
+  gg_status s = check_common((int64_t)E * mmax, K, N, E, masked_m, dev_status, &di);
+  if (s != GG_OK) return s;
+  if (W == nullptr) return GG_ERR_INVALID_ARG;
+  if (mmax == 0) return GG_OK;
+  if (A == nullptr || out == nullptr) return GG_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(W) || !aligned16(out)) return GG_ERR_UNSUPPORTED;
+  CUtensorMap ma, mb;
+  if (!map_2d(&ma, A, (int64_t)E * mmax, K, 64, gg::BM) || !map_w(&mb, W, E, K, N, 64, 64))
+    return GG_ERR_CUDA;
+  gg::Params p = base_params(masked_m, out, dev_status, (int64_t)E * mmax, E);
+  p.mmax = (int32_t)mmax;
+  p.red_len = (int32_t)K;
+  p.out_cols = (int32_t)N;
+  const int64_t tiles = (int64_t)E * cdiv(mmax, gg::BM) * cdiv(N, kBN);
+  return launch<Mode::Masked, kBN, kStages>(ma, mb, p, tiles, di, stream);
+}
+
+const char* gg_status_string(gg_status s) {
+  switch (s) {
+    case GG_OK: return "GG_OK";
+    case GG_ERR_INVALID_ARG: return "GG_ERR_INVALID_ARG: a pointer, size or count is invalid";
+    case GG_ERR_UNSUPPORTED:
+      return "GG_ERR_UNSUPPORTED: unsupported device, alignment, size or expert count";
+    case GG_ERR_CUDA: return "GG_ERR_CUDA: a CUDA runtime or driver call failed";
+  }
+  return "unknown gg_status";
+}
+
+uint64_t gg_set_watchdog_ns(uint64_t ns) {
+  return g_watchdog_ns.exchange(ns == 0 ? kDefaultWatchdogNs : ns);
+}
+
+int gg_testing_skip_first_load(int enable) { return g_skip_first_load.exchange(enable ? 1 : 0); }
+
+int gg_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,520 @@
+// Persistent, warp-specialised ragged grouped GEMM for sm_100a.
+//
+// One kernel template serves the four operations of the library:
+//   Forward  out[r,:]   = A[r,:] . W[e]                 (tile rows = token rows)
+//   Dgrad    dX[r,:]    = dY[r,:] . W[e]^T              (tile rows = token rows)
+//   Masked   out[e,r,:] = A[e,r,:] . W[e], r < masked_m[e]
+//   Wgrad    dW[e]      = A[rows of e]^T . dY[rows of e] (tile rows = K index; the reduction
+//                                                        runs over the ragged token rows)
+//
+// Roles of the 6 warps of a CTA (one CTA per SM, persistent over a strided tile list):
+//   warp 0      TMA producer: one lane arms a stage barrier and issues the tensor loads
+//   warp 1      tensor-memory owner and MMA issuer: one lane issues tcgen05.mma into a
+//               double-buffered fp32 accumulator in TMEM (2 x BN columns)
+//   warps 2..5  epilogue: tcgen05.ld of their 32-lane quadrant, fp32 -> bf16 (nearest even),
+//               predicated 16-byte stores of the rows inside the group and columns < N
+//
+// Shared-memory stages use the 128-byte swizzle that both TMA and tcgen05 understand:
+//   K-major operand  (reduction contiguous):  [rows][64 elements = 128 B]
+//   MN-major operand (M/N contiguous):        [chunks of 64 M/N][64 reduction rows][128 B]
+//
+// The tile list comes from the offsets on the device: every CTA rebuilds the same table
+// (group bounds under the clamp rule, tile prefix sums) in shared memory, so no host
+// synchronisation and no global scratch is needed. Every wait is bounded by a watchdog.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "ptx.cuh"
+
+namespace gg {
+
+enum class Mode : int { Forward = 0, Dgrad = 1, Wgrad = 2, Masked = 3 };
+
+constexpr int BM = 128;         // tile rows (TMEM lanes)
+constexpr int BK = 64;          // reduction elements per stage (128 bytes of bf16)
+constexpr int UMMA_K = 16;      // reduction per tcgen05.mma for 16-bit inputs
+constexpr int NUM_THREADS = 192;
+
+// Device status bits (same values as the public header).
+constexpr int DEV_BAD_OFFSETS = 0x1;
+constexpr int DEV_BAD_MASKED_M = 0x2;
+constexpr int DEV_TIMEOUT = 0x4;
+constexpr int DEV_LAUNCHED = 0x100;
+
+struct Params {
+  const int32_t* groups;   // offsets (ragged modes) or masked_m (masked mode), device
+  __nv_bfloat16* out;      // output base, row major with out_cols columns
+  int32_t* status;         // may be null
+  int64_t rows_alloc;      // rows of the token-major buffers (E*mmax in masked mode)
+  int32_t E;
+  int32_t mmax;            // masked mode only
+  int32_t red_len;         // reduction length (Forward/Masked: K, Dgrad: N; Wgrad: unused)
+  int32_t out_cols;        // output columns (Forward/Masked/Wgrad: N, Dgrad: K)
+  int32_t wg_K;            // Wgrad: K (rows of each dW[e])
+  uint64_t watchdog_ns;
+  int32_t debug_flags;     // bit 0: CTA 0 skips its first load (watchdog test)
+};
+
+template <int BN, int STAGES>
+struct Layout {
+  static constexpr uint32_t A_BYTES = BM * BK * 2;
+  static constexpr uint32_t B_BYTES = BN * BK * 2;
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t OFF_A = 0;
+  static constexpr uint32_t OFF_B = STAGES * A_BYTES;
+  static constexpr uint32_t OFF_BAR = STAGES * STAGE_BYTES;
+  static constexpr uint32_t NUM_BARS = 2 * STAGES + 5;  // full, empty, tfull x2, tempty x2, fin
+  static constexpr uint32_t OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr uint32_t OFF_TAB = OFF_MISC + 16;
+  static constexpr uint32_t TMEM_COLS = 2 * BN;
+  // gstart[E], gend[E], prefix[E+1], order[E] (int32)
+  static __host__ __device__ constexpr uint32_t bytes(int E) {
+    return OFF_TAB + 4u * (4u * (uint32_t)E + 1u) + 1024u /* alignment slack */;
+  }
+};
+
+struct Tile {
+  int32_t e;        // group / expert
+  int64_t row0;     // first output row of the tile (flat row of out)
+  int64_t row_end;  // rows >= row_end are not stored
+  int32_t n0;       // first output column
+  int32_t a_row0;   // token row of the first tile row (Forward/Dgrad/Masked)
+  int32_t k0;       // Wgrad: first K index of the tile
+  int32_t tok0;     // Wgrad: first token row of the group
+  int32_t tok_len;  // Wgrad: rows in the group
+  int32_t kblocks;  // reduction stages
+};
+
+struct Shared {
+  uint64_t* full;
+  uint64_t* empty;
+  uint64_t* tfull;
+  uint64_t* tempty;
+  uint64_t* fin;
+  uint32_t* tmem_base;
+  volatile int32_t* abort_flag;
+  int32_t* total;
+  int32_t* gstart;
+  int32_t* gend;
+  int32_t* prefix;
+  int32_t* order;
+};
+
+__device__ __forceinline__ void set_status(const Params& p, int bits) {
+  if (p.status != nullptr) atomicOr(p.status, bits);
+}
+
+// Bounded wait on one phase of an mbarrier. Returns false when the CTA is aborting or the
+// watchdog expired (then the abort flag and GG_DEV_TIMEOUT are set).
+__device__ __noinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, const Shared& sh,
+                                          const Params& p, bool honour_abort) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer();
+  for (uint32_t i = 1;; ++i) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if ((i & 31u) == 0u) {
+      if (honour_abort && *sh.abort_flag) return false;
+      if (ptx::globaltimer() - t0 > p.watchdog_ns) {
+        *sh.abort_flag = 1;
+        set_status(p, DEV_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// Single-lane wait whose outcome every lane of the warp shares.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const Shared& sh,
+                                          const Params& p) {
+  bool ok = true;
+  if (ptx::lane_id() == 0) ok = wait_bounded(bar, parity, sh, p, true);
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
+// ---------------------------------------------------------------- schedule
+// Warp 0 builds the group table. Ragged modes: effective ends t'_e = clamp(offs[e],
+// t'_{e-1}, rows_alloc) with t'_{-1} = 0, i.e. min(running max of offs (from 0), rows).
+// Masked: group e starts at e*mmax and has clamp(masked_m[e], 0, mmax) rows.
+template <Mode MODE, int BN>
+__device__ void build_table(const Params& p, const Shared& sh) {
+  const uint32_t lane = ptx::lane_id();
+  const int32_t E = p.E;
+  const int32_t NT = (p.out_cols + BN - 1) / BN;
+  int64_t run_max = 0;   // running max of offsets seen so far (starts at t'_{-1} = 0)
+  int32_t prev_end = 0;  // t'_{base-1}
+  int32_t tiles_carry = 0;
+  bool bad = false;
+  if (lane == 0) sh.prefix[0] = 0;
+  for (int32_t base = 0; base < E; base += 32) {
+    const int32_t e = base + (int32_t)lane;
+    const bool valid = e < E;
+    const int32_t g = valid ? p.groups[e] : 0;
+    int32_t start, end;
+    if constexpr (MODE == Mode::Masked) {
+      int32_t m = g < 0 ? 0 : (g > p.mmax ? p.mmax : g);
+      bad |= valid && (m != g);
+      start = e * p.mmax;
+      end = start + (valid ? m : 0);
+    } else {
+      int64_t v = valid ? (int64_t)g : INT64_MIN;
+      // inclusive max-scan across the warp
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int64_t o = __shfl_up_sync(0xffffffffu, v, d);
+        if ((int)lane >= d) v = v > o ? v : o;
+      }
+      v = v > run_max ? v : run_max;
+      const int64_t t = v < p.rows_alloc ? v : p.rows_alloc;
+      end = (int32_t)t;
+      const int32_t up = __shfl_up_sync(0xffffffffu, end, 1);
+      start = lane == 0 ? prev_end : up;
+      bad |= valid && ((int64_t)end != (int64_t)g);
+      run_max = __shfl_sync(0xffffffffu, v, 31);
+      prev_end = __shfl_sync(0xffffffffu, end, 31);
+    }
+    int32_t tiles = 0;
+    if (valid) {
+      if constexpr (MODE == Mode::Wgrad) {
+        tiles = 0;  // fixed grid, counted below
+      } else {
+        tiles = ((end - start + BM - 1) / BM) * NT;
+      }
+    }
+    int32_t s = tiles;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int32_t o = __shfl_up_sync(0xffffffffu, s, d);
+      if ((int)lane >= d) s += o;
+    }
+    if (valid) {
+      sh.gstart[e] = start;
+      sh.gend[e] = end;
+      sh.prefix[e + 1] = tiles_carry + s;
+    }
+    tiles_carry += __shfl_sync(0xffffffffu, s, 31);
+  }
+  bad = __any_sync(0xffffffffu, bad);
+  if (lane == 0) {
+    if (bad) set_status(p, MODE == Mode::Masked ? DEV_BAD_MASKED_M : DEV_BAD_OFFSETS);
+    if constexpr (MODE == Mode::Wgrad) {
+      const int32_t KT = (p.wg_K + BM - 1) / BM;
+      *sh.total = E * KT * NT;
+    } else {
+      *sh.total = tiles_carry;
+    }
+  }
+}
+
+// Wgrad visits experts in order of decreasing row count (ties by index) so that the
+// longest reductions start first; order[rank] = expert. All threads take part.
+__device__ void build_wgrad_order(const Params& p, const Shared& sh) {
+  const int32_t E = p.E;
+  for (int32_t e = threadIdx.x; e < E; e += blockDim.x) {
+    const int32_t me = sh.gend[e] - sh.gstart[e];
+    int32_t rank = 0;
+    for (int32_t j = 0; j < E; ++j) {
+      const int32_t mj = sh.gend[j] - sh.gstart[j];
+      rank += (mj > me) || (mj == me && j < e);
+    }
+    sh.order[rank] = e;
+  }
+}
+
+template <Mode MODE, int BN>
+__device__ __forceinline__ Tile decode_tile(int32_t t, const Params& p, const Shared& sh) {
+  Tile tl;
+  const int32_t NT = (p.out_cols + BN - 1) / BN;
+  if constexpr (MODE == Mode::Wgrad) {
+    const int32_t KT = (p.wg_K + BM - 1) / BM;
+    const int32_t per = KT * NT;
+    const int32_t slot = t / per;
+    const int32_t local = t - slot * per;
+    const int32_t kt = local / NT;
+    const int32_t nt = local - kt * NT;
+    const int32_t e = sh.order[slot];
+    tl.e = e;
+    tl.k0 = kt * BM;
+    tl.n0 = nt * BN;
+    tl.tok0 = sh.gstart[e];
+    tl.tok_len = sh.gend[e] - sh.gstart[e];
+    tl.kblocks = (tl.tok_len + BK - 1) / BK;
+    tl.row0 = (int64_t)e * p.wg_K + tl.k0;
+    tl.row_end = (int64_t)e * p.wg_K + p.wg_K;
+    tl.a_row0 = 0;
+  } else {
+    // largest e with prefix[e] <= t
+    int32_t lo = 0, hi = p.E - 1;
+    while (lo < hi) {
+      const int32_t mid = (lo + hi + 1) >> 1;
+      if (sh.prefix[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    const int32_t e = lo;
+    const int32_t local = t - sh.prefix[e];
+    const int32_t mt = local / NT;
+    const int32_t nt = local - mt * NT;
+    tl.e = e;
+    tl.a_row0 = sh.gstart[e] + mt * BM;
+    tl.row0 = tl.a_row0;
+    tl.row_end = sh.gend[e];
+    tl.n0 = nt * BN;
+    tl.kblocks = (p.red_len + BK - 1) / BK;
+    tl.k0 = 0;
+    tl.tok0 = 0;
+    tl.tok_len = 0;
+  }
+  return tl;
+}
+
+// ---------------------------------------------------------------- kernel
+template <Mode MODE, int BN, int STAGES>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap mapA,
+                        const __grid_constant__ CUtensorMap mapB, const Params p) {
+  using L = Layout<BN, STAGES>;
+  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN must be 64, 128, 192 or 256");
+  static_assert(L::TMEM_COLS == 128 || L::TMEM_COLS == 256 || L::TMEM_COLS == 512,
+                "TMEM allocation must be a power of two");
+  // A operand MN-major only in Wgrad; B operand K-major only in Dgrad.
+  constexpr uint32_t A_MN = (MODE == Mode::Wgrad) ? 1u : 0u;
+  constexpr uint32_t B_MN = (MODE == Mode::Dgrad) ? 0u : 1u;
+  constexpr uint32_t IDESC = ptx::idesc_bf16_f32(BM, BN, A_MN, B_MN);
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = ptx::smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+
+  Shared sh;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  sh.full = bars;
+  sh.empty = bars + STAGES;
+  sh.tfull = bars + 2 * STAGES;
+  sh.tempty = bars + 2 * STAGES + 2;
+  sh.fin = bars + 2 * STAGES + 4;
+  sh.tmem_base = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  sh.abort_flag = reinterpret_cast<volatile int32_t*>(smem + L::OFF_MISC + 4);
+  sh.total = reinterpret_cast<int32_t*>(smem + L::OFF_MISC + 8);
+  int32_t* tab = reinterpret_cast<int32_t*>(smem + L::OFF_TAB);
+  sh.gstart = tab;
+  sh.gend = tab + p.E;
+  sh.prefix = tab + 2 * p.E;
+  sh.order = tab + 3 * p.E + 1;
+
+  const uint32_t warp = threadIdx.x / 32;
+  const uint32_t lane = ptx::lane_id();
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      ptx::mbar_init(&sh.full[s], 1);
+      ptx::mbar_init(&sh.empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      ptx::mbar_init(&sh.tfull[a], 1);
+      ptx::mbar_init(&sh.tempty[a], 128);
+    }
+    ptx::mbar_init(sh.fin, 1);
+    *sh.abort_flag = 0;
+    ptx::fence_mbar_init();
+    ptx::prefetch_tmap(&mapA);
+    ptx::prefetch_tmap(&mapB);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(sh.tmem_base, L::TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  if (warp == 0) build_table<MODE, BN>(p, sh);
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if constexpr (MODE == Mode::Wgrad) {
+    build_wgrad_order(p, sh);
+    __syncthreads();
+  }
+  const uint32_t tmem_base = *sh.tmem_base;
+  const int32_t total = *sh.total;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_stream = ptx::policy_evict_first();
+      const uint64_t pol_keep = ptx::policy_evict_last();
+      uint32_t stage = 0, phase = 0;
+      uint32_t armed = 0, armed_par = 0;  // per-stage: loads in flight, and their phase
+      bool skip_first = (p.debug_flags & 1) && blockIdx.x == 0;
+      bool ok = true;
+      for (int32_t t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const Tile tl = decode_tile<MODE, BN>(t, p, sh);
+        for (int32_t kb = 0; kb < tl.kblocks; ++kb) {
+          if (!wait_bounded(&sh.empty[stage], phase ^ 1u, sh, p, true)) { ok = false; break; }
+          armed &= ~(1u << stage);
+          uint8_t* sA = smem + L::OFF_A + stage * L::A_BYTES;
+          uint8_t* sB = smem + L::OFF_B + stage * L::B_BYTES;
+          uint64_t* fb = &sh.full[stage];
+          if (skip_first) {
+            skip_first = false;  // watchdog test: never arm this stage
+          } else {
+            ptx::mbar_arrive_expect_tx(fb, L::STAGE_BYTES);
+            if constexpr (MODE == Mode::Forward || MODE == Mode::Masked) {
+              ptx::tma_load_2d(sA, &mapA, fb, kb * BK, tl.a_row0, pol_stream);
+#pragma unroll
+              for (int j = 0; j < BN / 64; ++j)
+                ptx::tma_load_3d(sB + j * 8192, &mapB, fb, tl.n0 + j * 64, kb * BK, tl.e,
+                                 pol_keep);
+            } else if constexpr (MODE == Mode::Dgrad) {
+              ptx::tma_load_2d(sA, &mapA, fb, kb * BK, tl.a_row0, pol_stream);
+              ptx::tma_load_3d(sB, &mapB, fb, kb * BK, tl.n0, tl.e, pol_keep);
+            } else {  // Wgrad
+              const int32_t r = tl.tok0 + kb * BK;
+#pragma unroll
+              for (int j = 0; j < 2; ++j)
+                ptx::tma_load_2d(sA + j * 8192, &mapA, fb, tl.k0 + j * 64, r, pol_keep);
+#pragma unroll
+              for (int j = 0; j < BN / 64; ++j)
+                ptx::tma_load_2d(sB + j * 8192, &mapB, fb, tl.n0 + j * 64, r, pol_keep);
+            }
+            armed |= 1u << stage;
+            armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+          }
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // Let every load this thread issued land before the CTA can exit (on the normal path
+      // these phases have completed already; after an abort some may still be in flight).
+      for (int s = 0; s < STAGES; ++s)
+        if (armed & (1u << s)) wait_bounded(&sh.full[s], (armed_par >> s) & 1u, sh, p, false);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    uint32_t stage = 0, phase = 0, acc_iter = 0;
+    bool ok = true;
+    for (int32_t t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      const Tile tl = decode_tile<MODE, BN>(t, p, sh);
+      if (tl.kblocks == 0) continue;  // Wgrad of an empty expert: the epilogue writes zeros
+      const uint32_t a = acc_iter & 1u;
+      if (!warp_wait(&sh.tempty[a], ((acc_iter >> 1) & 1u) ^ 1u, sh, p)) { ok = false; break; }
+      ptx::tc_fence_after();
+      const uint32_t d_tmem = tmem_base + a * BN;
+      for (int32_t kb = 0; kb < tl.kblocks; ++kb) {
+        if (!warp_wait(&sh.full[stage], phase, sh, p)) { ok = false; break; }
+        ptx::tc_fence_after();
+        uint8_t* sA = smem + L::OFF_A + stage * L::A_BYTES;
+        uint8_t* sB = smem + L::OFF_B + stage * L::B_BYTES;
+        int nsub = BK / UMMA_K;
+        if constexpr (MODE == Mode::Wgrad) {
+          const int32_t rem = tl.tok_len - kb * BK;  // rows of this group in the stage
+          if (rem < BK) {
+            nsub = (rem + UMMA_K - 1) / UMMA_K;
+            // Rows [rem, nsub*16) belong to the next group (or to no group): zero them in
+            // both operands so they add nothing. Each token row is one 128-byte line of
+            // every 64-wide chunk.
+            const int zrows = nsub * UMMA_K - rem;
+            const int lines_a = zrows * 2, lines_b = zrows * (BN / 64);
+            for (int i = (int)lane; i < (lines_a + lines_b) * 8; i += 32) {
+              const int line = i >> 3, part = i & 7;
+              uint8_t* dst;
+              if (line < lines_a) {
+                const int c = line / zrows, rr = rem + line % zrows;
+                dst = sA + c * 8192 + rr * 128 + part * 16;
+              } else {
+                const int l2 = line - lines_a;
+                const int c = l2 / zrows, rr = rem + l2 % zrows;
+                dst = sB + c * 8192 + rr * 128 + part * 16;
+              }
+              *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+            }
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+          }
+        }
+        if (lane == 0) {
+          const uint32_t a_base = ptx::smem_u32(sA), b_base = ptx::smem_u32(sB);
+          for (int k = 0; k < nsub; ++k) {
+            uint64_t adesc, bdesc;
+            if constexpr (A_MN) adesc = ptx::smem_desc_sw128(a_base + k * 2048, 8192, 1024);
+            else                adesc = ptx::smem_desc_sw128(a_base + k * 32, 16, 1024);
+            if constexpr (B_MN) bdesc = ptx::smem_desc_sw128(b_base + k * 2048, 8192, 1024);
+            else                bdesc = ptx::smem_desc_sw128(b_base + k * 32, 16, 1024);
+            ptx::mma_bf16(d_tmem, adesc, bdesc, IDESC, (kb > 0 || k > 0) ? 1u : 0u);
+          }
+          ptx::mma_commit(&sh.empty[stage]);  // frees the stage once these MMAs are done
+        }
+        __syncwarp();
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+      if (lane == 0) ptx::mma_commit(&sh.tfull[a]);
+      __syncwarp();
+      ++acc_iter;
+    }
+    // every MMA issued by this CTA completes before tensor memory is released
+    if (lane == 0) {
+      ptx::mma_commit(sh.fin);
+      wait_bounded(sh.fin, 0, sh, p, false);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const uint32_t q = warp & 3u;  // TMEM lane quadrant this warp may access
+    const int32_t row_in_tile = (int32_t)(q * 32 + lane);
+    uint32_t acc_iter = 0;
+    for (int32_t t = blockIdx.x; t < total; t += gridDim.x) {
+      const Tile tl = decode_tile<MODE, BN>(t, p, sh);
+      const int64_t orow = tl.row0 + row_in_tile;
+      const bool row_ok = orow < tl.row_end;
+      __nv_bfloat16* orow_ptr = p.out + orow * (int64_t)p.out_cols;
+      if (tl.kblocks == 0) {
+        if (row_ok) {
+          for (int c = 0; c < BN; c += 8) {
+            const int32_t col = tl.n0 + c;
+            if (col < p.out_cols)
+              *reinterpret_cast<uint4*>(orow_ptr + col) = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+        continue;
+      }
+      const uint32_t a = acc_iter & 1u;
+      if (!warp_wait(&sh.tfull[a], (acc_iter >> 1) & 1u, sh, p)) break;
+      ptx::tc_fence_after();
+      const uint32_t taddr = tmem_base + ((q * 32u) << 16) + a * BN;
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t r[32];
+        ptx::tmem_ld_32x32b_x32(taddr + c, r);
+        ptx::tmem_ld_wait();
+        if (row_ok) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int32_t col = tl.n0 + c + j * 8;
+            if (col < p.out_cols) {
+              uint4 v;
+              uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[j * 8 + 2 * h]),
+                                                          __uint_as_float(r[j * 8 + 2 * h + 1]));
+                w[h] = *reinterpret_cast<uint32_t*>(&b2);
+              }
+              *reinterpret_cast<uint4*>(orow_ptr + col) = v;
+            }
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&sh.tempty[a]);
+      ++acc_iter;
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, L::TMEM_COLS);
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0 && !*sh.abort_flag) set_status(p, DEV_LAUNCHED);
+}
+
+}  // namespace gg

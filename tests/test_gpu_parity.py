@@ -1,0 +1,163 @@
+"""Parity of the sm_100a kernels (through the C ABI) with the CPU oracle.
+
+Every comparison is elementwise against the fp64 oracle on the same seeded inputs with
+|gpu - ref| <= 1e-2*|ref| + 1e-2; group membership and untouched regions are bit-exact
+(sentinel bit patterns), and so are the exact zeros of an empty expert's wgrad.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from conftest import cuda_ok
+from helpers import assert_close, is_sentinel, sample_k, sample_rows, sentinel, to_f64
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not cuda_ok(), reason="needs a CUDA device")]
+
+gg = pytest.importorskip("moe_grouped_gemm_ragged_b200")
+
+
+def _dev(r: workloads.RaggedInputs):
+    return (r.A.cuda(), r.W.cuda(), r.dY.cuda(),
+            torch.from_numpy(np.ascontiguousarray(r.offs)).cuda())
+
+
+def run_ragged(r: workloads.RaggedInputs):
+    """All three passes on the GPU into sentinel-filled buffers; returns device tensors."""
+    A, W, dY, offs = _dev(r) if r.A.device.type == "cpu" else (
+        r.A, r.W, r.dY, torch.from_numpy(np.ascontiguousarray(r.offs)).cuda())
+    rows, K, N, E = r.rows_alloc, r.K, r.N, r.E
+    out = sentinel((rows, N))
+    dX = sentinel((rows, K))
+    dW = sentinel((E, K, N))
+    st = torch.zeros(3, dtype=torch.int32, device="cuda")
+    gg.forward(A, W, offs, out, status=st[0:1])
+    gg.dgrad(dY, W, offs, dX, status=st[1:2])
+    gg.wgrad(A, dY, offs, dW, status=st[2:3])
+    torch.cuda.synchronize()
+    return out, dX, dW, st.cpu().numpy()
+
+
+def check_ragged(r: workloads.RaggedInputs, sample: bool, seed: int = 0,
+                 expect_status: int = 0):
+    out, dX, dW, st = run_ragged(r)
+    for s in st:
+        assert s & gg.DEV_LAUNCHED, "the sm_100a kernel did not report completion"
+        assert (s & gg.DEV_ERROR_MASK) == expect_status, hex(s)
+    A, W, dY = oracle.as_u16(r.A), oracle.as_u16(r.W), oracle.as_u16(r.dY)  # host copies
+    rows = sample_rows(r.offs, r.rows_alloc, seed) if sample else None
+    ref, grp = oracle.forward(A, W, r.offs, rows=rows)
+    sel = grp >= 0
+    ridx = np.arange(r.rows_alloc) if rows is None else rows
+    ridx_t = torch.from_numpy(ridx[sel]).cuda()
+    assert_close(to_f64(out.index_select(0, ridx_t)), ref[sel], "forward")
+    refd, _ = oracle.dgrad(dY, W, r.offs, rows=rows)
+    assert_close(to_f64(dX.index_select(0, ridx_t)), refd[sel], "dgrad")
+    # rows outside every group: untouched, bit for bit
+    untouched = torch.from_numpy(oracle.untouched_rows(r.offs, r.rows_alloc)).cuda()
+    assert bool(is_sentinel(out.index_select(0, untouched)).all())
+    assert bool(is_sentinel(dX.index_select(0, untouched)).all())
+    ks = sample_k(r.K, seed) if sample else None
+    refw = oracle.wgrad(A, dY, r.offs, ks=ks)
+    kidx = torch.from_numpy(np.arange(r.K) if ks is None else ks).cuda()
+    assert_close(to_f64(dW.index_select(1, kidx)), refw, "wgrad")
+    # every dW element written; an empty expert's dW is exactly +0.0
+    assert not bool(is_sentinel(dW).any())
+    starts, ends, _ = oracle.group_bounds(r.offs, r.rows_alloc)
+    for e in np.nonzero(ends == starts)[0]:
+        assert bool((dW[e].view(torch.int16) == 0).all()), f"dW[{e}] of an empty expert"
+    return out, dX, dW
+
+
+@pytest.mark.parametrize("offs", [(8, 16, 32, 40), (8, 8, 32, 40), (0, 16, 32, 40),
+                                  (8, 16, 32, 32), (0, 0, 0, 0), (40, 40, 40, 40),
+                                  (48, 48, 48, 48), (0, 0, 0, 48)])
+def test_tiny_repro_offsets(offs):
+    """The 4-expert M=48/K=8/N=16 repro with its two offset tuples and edge variants."""
+    r = workloads.make_tiny(offs)
+    out, dX, dW = check_ragged(r, sample=False)
+    assert tuple(out.shape) == (48, 16) and tuple(dX.shape) == (48, 8)
+    assert tuple(dW.shape) == (4, 8, 16)
+
+
+SWEEP = [0, 1, 7, 8, 9, 15, 16, 17, 127, 128, 129, 255, 256, 257]
+
+
+@pytest.mark.parametrize("K,N", [(200, 328), (64, 256), (8, 16), (136, 520)])
+def test_group_size_sweep(K, N):
+    """Group sizes around 0, 8, 16, 128 and 256 rows, K and N tails, NaN tail rows."""
+    r = workloads.make_ragged_custom(len(SWEEP), K, N, SWEEP, seed=100 + K, tail=128)
+    check_ragged(r, sample=False)
+
+
+def test_shuffled_sizes_many_experts():
+    rng = np.random.default_rng(7)
+    sizes = rng.permutation(np.array(SWEEP * 3))
+    r = workloads.make_ragged_custom(len(sizes), 256, 384, sizes, seed=8, tail=200)
+    check_ragged(r, sample=False)
+
+
+def test_group_id_probe_bit_exact():
+    """A[:,0]=1, W[e][0,:]=e+1: every output row equals its group id + 1 exactly."""
+    sizes = [3, 0, 130, 1, 257, 0, 64]
+    E, K, N = len(sizes), 64, 264
+    offs = workloads.offsets_from_sizes(sizes)
+    rows = int(offs[-1]) + 16
+    A = torch.zeros(rows, K, dtype=torch.bfloat16)
+    A[:, 0] = 1
+    W = torch.zeros(E, K, N, dtype=torch.bfloat16)
+    for e in range(E):
+        W[e, 0] = e + 1
+    out = sentinel((rows, N))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    gg.forward(A.cuda(), W.cuda(), torch.from_numpy(offs).cuda(), out, status=st)
+    torch.cuda.synchronize()
+    grp = np.concatenate([np.full(s, e) for e, s in enumerate(sizes)])
+    expect = torch.from_numpy(grp + 1).float().cuda()[:, None].expand(-1, N)
+    assert bool((out[: int(offs[-1])].float() == expect).all())
+    assert bool(is_sentinel(out[int(offs[-1]):]).all())
+
+
+def test_masked_config_full():
+    """Masked layout E=8, mmax=128, K=768, N=2048; NaN in inactive rows."""
+    m = workloads.make_masked()
+    A, W = m.A.cuda(), m.W.cuda()
+    mm = torch.from_numpy(m.masked_m).cuda()
+    out = sentinel((m.E, m.mmax, m.N))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    gg.masked_forward(A, W, mm, out, status=st)
+    torch.cuda.synchronize()
+    s = int(st.item())
+    assert s & gg.DEV_LAUNCHED and (s & gg.DEV_ERROR_MASK) == 0
+    ref, act, _ = oracle.masked_forward(m.A, m.W, m.masked_m)
+    flat = out.view(-1, m.N)
+    act_t = torch.from_numpy(np.nonzero(act)[0]).cuda()
+    inact_t = torch.from_numpy(np.nonzero(~act)[0]).cuda()
+    assert_close(to_f64(flat.index_select(0, act_t)), ref[act], "masked forward")
+    assert bool(is_sentinel(flat.index_select(0, inact_t)).all())
+
+
+@pytest.mark.parametrize("name", ["gateup", "downproj"])
+def test_moe_projection_configs(name):
+    """E=64 Zipf gate-up (K=2048, N=1536) and E=32 down-proj (K=2048, N=7168): sampled rows
+    {s, s+1, t-2, t-1} + 60 random per group and 32 K rows per expert, NaN tail rows."""
+    r = workloads.make_ragged(name, tail=128, device="cuda")
+    check_ragged(r, sample=True, seed=1)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["large", "large_unaligned"])
+def test_large_configs(name):
+    """262144 x 6144 x 4096, E=16, aligned and +-1..127 perturbed sizes (sampled)."""
+    r = workloads.make_ragged(name, tail=128, device="cuda")
+    check_ragged(r, sample=True, seed=2)
+
+
+def test_repeat_calls_bit_identical():
+    r = workloads.make_ragged_custom(5, 192, 512, [100, 0, 300, 7, 513], seed=3, tail=9)
+    a = run_ragged(r)
+    b = run_ragged(r)
+    for x, y in zip(a[:3], b[:3]):
+        assert bool((x.view(torch.int16) == y.view(torch.int16)).all())
