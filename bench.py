@@ -1,0 +1,407 @@
+"""Benchmark of the ragged MoE grouped GEMM on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+forward, dgrad and wgrad of the large grouped GEMM (E=16, T=262144 rows, K=6144, N=4096,
+bf16, the TileOPs issue 1566 "GLM-up" shape) plus the masked forward of the sglang PR 32385
+shape (E=8, mmax=128, K=768, N=2048). The metric is grouped GEMM bf16 TFLOP/s with
+algorithmic flops 2*T*K*N per pass (T counts real rows only).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs its own copy of the per-GPU workload (expert
+parallelism: each GPU owns its experts; no collective on the data path), the timed region
+is bracketed by barriers, and rank 0 prints the max-over-ranks time. ``--impl reference``
+times the CPU oracle on a bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "grouped GEMM BF16 TFLOP/s (fwd/dgrad/wgrad) and % of B200 dense BF16 peak"
+UNIT = "TFLOP/s"
+
+# DRAM bytes per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum), keyed by
+# kernel and workload, valid only for the kernel sources whose hash is recorded with them.
+NCU_TRAFFIC = {}
+NCU_TRAFFIC_SRC_HASH = None
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "moe_grouped_gemm_ragged_b200", "csrc", "*"))):
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, \
+        "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.lines = []
+        sel = str(device_index)
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            pass
+        self.sel = sel
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.sel, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        loaded = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def workload_desc(name, r, m) -> str:
+    return (f"{name}: E={r.E} T={r.T} K={r.K} N={r.N} bf16 (fwd+dgrad+wgrad) + masked "
+            f"E={m.E} mmax={m.mmax} K={m.K} N={m.N} fwd")
+
+
+def make_inputs(workload: str, device):
+    import workloads
+    r = workloads.make_ragged(workload, tail=0, device=device)
+    m = workloads.make_masked(device=device)
+    return r, m
+
+
+def oracle_sample_step(r, m, host, rows_per_group: int, k_per_expert: int, threads: int):
+    """One bounded oracle step: forward/dgrad on sampled rows, wgrad on sampled K rows,
+    masked forward on all its rows. Returns (flops, seconds)."""
+    import oracle
+    A, W, dY = host["A"], host["W"], host["dY"]
+    rng = np.random.default_rng(0)
+    starts, ends, _ = oracle.group_bounds(r.offs, r.rows_alloc)
+    rows = np.concatenate([rng.integers(s, t, rows_per_group) for s, t in zip(starts, ends)
+                           if t > s]).astype(np.int64)
+    ks = np.sort(rng.choice(r.K, k_per_expert, replace=False)).astype(np.int64)
+    t0 = time.perf_counter()
+    oracle.forward(A, W, r.offs, rows=rows, threads=threads)
+    oracle.dgrad(dY, W, r.offs, rows=rows, threads=threads)
+    oracle.wgrad(A, dY, r.offs, ks=ks, threads=threads)
+    oracle.masked_forward(host["mA"], host["mW"], m.masked_m, threads=threads)
+    dt = time.perf_counter() - t0
+    flops = (2 * 2 * len(rows) * r.K * r.N + 2 * int(r.sizes.sum()) * len(ks) * r.N
+             + m.flops)
+    sample = (f"forward+dgrad on {rows_per_group} random rows per group, wgrad on "
+              f"{k_per_expert} random K rows of every expert, full masked forward")
+    return flops, dt, sample
+
+
+def host_copies(r, m):
+    import oracle
+    return {"A": oracle.as_u16(r.A), "W": oracle.as_u16(r.W), "dY": oracle.as_u16(r.dY),
+            "mA": oracle.as_u16(m.A), "mW": oracle.as_u16(m.W)}
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    threads = oracle.default_threads()
+    r, m = make_inputs(args.workload, "cpu")
+    host = host_copies(r, m)
+    for _ in range(args.warmup):
+        oracle_sample_step(r, m, host, 16, 8, threads)
+    flops = secs = 0.0
+    sample = ""
+    for _ in range(args.steps):
+        f, dt, sample = oracle_sample_step(r, m, host, 16, 8, threads)
+        flops += f
+        secs += dt
+    value = flops / secs / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * secs / max(args.steps, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(args.workload, r, m), "parallelism": "cpu oracle"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import moe_grouped_gemm_ragged_b200 as gg
+
+    ws, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (there is no CPU implementation)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+
+    def barrier():
+        if ws > 1:
+            torch.distributed.barrier()
+
+    r, m = make_inputs(args.workload, dev)
+    rows, K, N, E = r.rows_alloc, r.K, r.N, r.E
+    offs = torch.from_numpy(r.offs).to(dev)
+    mm = torch.from_numpy(m.masked_m).to(dev)
+    out = torch.empty((rows, N), dtype=torch.bfloat16, device=dev)
+    dX = torch.empty((rows, K), dtype=torch.bfloat16, device=dev)
+    dW = torch.empty((E, K, N), dtype=torch.bfloat16, device=dev)
+    mout = torch.empty((m.E, m.mmax, m.N), dtype=torch.bfloat16, device=dev)
+    status = torch.zeros(4, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    passes = ["forward", "dgrad", "wgrad", "masked"]
+    pass_flops = [r.flops, r.flops, r.flops, m.flops]
+    step_flops = sum(pass_flops)
+
+    def step(evs=None):
+        if evs is not None:
+            evs[0].record(stream)
+        gg.forward(r.A, r.W, offs, out, status=status[0:1])
+        if evs is not None:
+            evs[1].record(stream)
+        gg.dgrad(r.dY, r.W, offs, dX, status=status[1:2])
+        if evs is not None:
+            evs[2].record(stream)
+        gg.wgrad(r.A, r.dY, offs, dW, status=status[2:3])
+        if evs is not None:
+            evs[3].record(stream)
+        gg.masked_forward(m.A, m.W, mm, mout, status=status[3:4])
+        if evs is not None:
+            evs[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = status.cpu().numpy()
+    if np.any(st & gg.DEV_ERROR_MASK) or not np.all(st & gg.DEV_LAUNCHED):
+        raise SystemExit(f"kernel status after warm-up: {[hex(x) for x in st]}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    per_pass_ms = [sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
+                   / args.steps for j in range(4)]
+    if ws > 1:
+        t = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = ws * step_flops / (ms_per_step * 1e-3) / 1e12
+
+    # end to end through the public API: pinned host inputs -> device, all passes, results
+    # back to pinned host memory, every step inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, gg, r, m, dev, stream, ws, barrier)
+
+    peaks, peak_src = load_peaks()
+    dom = int(np.argmax(per_pass_ms[:3]))
+    dom_tflops = pass_flops[dom] / (per_pass_ms[dom] * 1e-3) / 1e12
+    peak_sus = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    traffic = None
+    if NCU_TRAFFIC_SRC_HASH == kernel_source_hash():
+        traffic = NCU_TRAFFIC.get((passes[dom], args.workload))
+    roofline = {"bound": "tensor", "kernel": f"grouped_gemm_kernel<{passes[dom]}>",
+                "achieved": dom_tflops, "peak": peak_sus, "unit": "TFLOP/s",
+                "frac": dom_tflops / peak_sus, "traffic": traffic,
+                "peak_kind": f"bf16_tflops_sustained ({peak_src}): the kernel runs inside a "
+                             "seconds-long back-to-back timed region",
+                "frac_of_burst_peak": dom_tflops / peaks["bf16_tflops"],
+                "frac_of_spec_2250": dom_tflops / 2250.0}
+
+    cpu = None
+    if rank == 0 and not args.no_cpu:
+        import oracle
+        threads = oracle.default_threads()
+        host = host_copies(r, m)
+        f, dt, sample = oracle_sample_step(r, m, host, 32, 16, threads)
+        cpu = {"value": f / dt / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": sample, "seconds": dt}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {
+                "workload": workload_desc(args.workload, r, m),
+                "group_sizes": f"min {int(r.sizes.min())} max {int(r.sizes.max())}",
+                "l2": "inputs (>6 GB) exceed the 126 MB L2; no flush",
+                "parallelism": f"ep{ws} (independent per-GPU experts)",
+            },
+            "passes": {p: {"ms": per_pass_ms[j],
+                           "tflops": pass_flops[j] / (per_pass_ms[j] * 1e-3) / 1e12}
+                       for j, p in enumerate(passes)},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": 4 * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def run_e2e(args, gg, r, m, dev, stream, ws, barrier):
+    steps = max(1, min(args.steps, args.e2e_steps))
+    hA = r.A.cpu().pin_memory()
+    hW = r.W.cpu().pin_memory()
+    hdY = r.dY.cpu().pin_memory()
+    hoffs = torch.from_numpy(r.offs).pin_memory()
+    hmA, hmW = m.A.cpu().pin_memory(), m.W.cpu().pin_memory()
+    hmm = torch.from_numpy(m.masked_m).pin_memory()
+    rows, K, N, E = r.rows_alloc, r.K, r.N, r.E
+    dA = torch.empty_like(r.A)
+    dWt = torch.empty_like(r.W)
+    ddY = torch.empty_like(r.dY)
+    doffs = torch.empty(E, dtype=torch.int32, device=dev)
+    dmA, dmW = torch.empty_like(m.A), torch.empty_like(m.W)
+    dmm = torch.empty(m.E, dtype=torch.int32, device=dev)
+    out = torch.empty((rows, N), dtype=torch.bfloat16, device=dev)
+    dX = torch.empty((rows, K), dtype=torch.bfloat16, device=dev)
+    dW = torch.empty((E, K, N), dtype=torch.bfloat16, device=dev)
+    mout = torch.empty((m.E, m.mmax, m.N), dtype=torch.bfloat16, device=dev)
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    hdX = torch.empty(dX.shape, dtype=dX.dtype).pin_memory()
+    hdW = torch.empty(dW.shape, dtype=dW.dtype).pin_memory()
+    hmout = torch.empty(mout.shape, dtype=mout.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (hA, hW, hdY, hoffs, hmA, hmW, hmm))
+    d2h = sum(t.numel() * t.element_size() for t in (hout, hdX, hdW, hmout))
+
+    def step():
+        for d, h in ((dA, hA), (dWt, hW), (ddY, hdY), (doffs, hoffs), (dmA, hmA), (dmW, hmW),
+                     (dmm, hmm)):
+            d.copy_(h, non_blocking=True)
+        gg.forward(dA, dWt, doffs, out)
+        gg.dgrad(ddY, dWt, doffs, dX)
+        gg.wgrad(dA, ddY, doffs, dW)
+        gg.masked_forward(dmA, dmW, dmm, mout)
+        for h, d in ((hout, out), (hdX, dX), (hdW, dW), (hmout, mout)):
+            h.copy_(d, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = e0.elapsed_time(e1) / steps
+    if ws > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    flops = 3 * r.flops + m.flops
+    return {"value": ws * flops / (ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms,
+            "steps": steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="large",
+                    choices=["large", "large_unaligned", "gateup", "downproj"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
