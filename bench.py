@@ -206,6 +206,7 @@ def run_ours(args):
         if ws > 1:
             torch.distributed.barrier()
 
+    gg.testing_force_variant(args.variant)
     r, m = make_inputs(args.workload, dev)
     rows, K, N, E = r.rows_alloc, r.K, r.N, r.E
     offs = torch.from_numpy(r.offs).to(dev)
@@ -395,6 +396,8 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--variant", type=int, default=0, choices=[0, 1, 2],
+                    help="launch shape of forward/dgrad: 0 automatic, 1 single CTA, 2 CTA pair")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3

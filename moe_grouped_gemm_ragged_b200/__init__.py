@@ -61,6 +61,8 @@ def lib() -> ctypes.CDLL:
     L.gg_set_watchdog_ns.restype = ctypes.c_uint64
     L.gg_testing_skip_first_load.argtypes = [ctypes.c_int]
     L.gg_testing_skip_first_load.restype = ctypes.c_int
+    L.gg_testing_force_variant.argtypes = [ctypes.c_int]
+    L.gg_testing_force_variant.restype = ctypes.c_int
     L.gg_version.restype = ctypes.c_int
     _lib = L
     return L
@@ -82,6 +84,11 @@ def set_watchdog_ns(ns: int) -> int:
 def testing_skip_first_load(enable: bool) -> bool:
     """Test hook: make later calls' first load go missing so the watchdog fires."""
     return bool(lib().gg_testing_skip_first_load(1 if enable else 0))
+
+
+def testing_force_variant(variant: int) -> int:
+    """Test hook: 0 automatic, 1 single-CTA tiles, 2 CTA-pair tiles (forward and dgrad)."""
+    return int(lib().gg_testing_force_variant(int(variant)))
 
 
 def _stream_handle(stream) -> int:
@@ -209,7 +216,7 @@ def grouped_mm(A: torch.Tensor, W: torch.Tensor, offs: torch.Tensor,
 
 __all__ = [
     "forward", "dgrad", "wgrad", "masked_forward", "grouped_mm", "status_string", "version",
-    "set_watchdog_ns", "testing_skip_first_load", "lib", "GGError", "LIB_PATH",
+    "set_watchdog_ns", "testing_skip_first_load", "testing_force_variant", "lib", "GGError", "LIB_PATH",
     "DEV_BAD_OFFSETS", "DEV_BAD_MASKED_M", "DEV_TIMEOUT", "DEV_ERROR_MASK", "DEV_LAUNCHED",
     "MAX_EXPERTS",
 ]

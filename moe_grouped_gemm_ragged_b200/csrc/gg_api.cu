@@ -23,6 +23,7 @@ constexpr uint64_t kDefaultWatchdogNs = 4000000000ull;
 
 std::atomic<uint64_t> g_watchdog_ns{kDefaultWatchdogNs};
 std::atomic<int> g_skip_first_load{0};
+std::atomic<int> g_force_variant{0};  // test hook: 0 automatic, 1 single CTA, 2 CTA pair
 
 static_assert(gg::DEV_BAD_OFFSETS == GG_DEV_BAD_OFFSETS, "status bit mismatch");
 static_assert(gg::DEV_BAD_MASKED_M == GG_DEV_BAD_MASKED_M, "status bit mismatch");
@@ -114,28 +115,66 @@ bool map_w(CUtensorMap* m, const void* W, int64_t E, int64_t K, int64_t N, uint3
   return make_map(m, W, 3, dims, str, box);
 }
 
-template <Mode MODE, int BN, int STAGES>
+template <Mode MODE, int BN, int STAGES, bool PAIR>
 gg_status launch(const CUtensorMap& a, const CUtensorMap& b, const gg::Params& p,
                  int64_t tiles_upper, const DeviceInfo& di, cudaStream_t stream) {
-  auto kern = gg::grouped_gemm_kernel<MODE, BN, STAGES>;
-  const size_t smem = gg::Layout<BN, STAGES>::bytes(p.E);
+  auto kern = gg::grouped_gemm_kernel<MODE, BN, STAGES, PAIR>;
+  using L = gg::Layout<BN, STAGES, PAIR>;
+  const size_t smem = L::bytes(p.E);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return GG_ERR_CUDA;
   static bool attr_done[kMaxDevices] = {};
+  static int max_units[kMaxDevices] = {};
   static std::mutex mu;
   {
     std::lock_guard<std::mutex> lk(mu);
     if (!attr_done[dev]) {
-      const int max_smem = (int)gg::Layout<BN, STAGES>::bytes(GG_MAX_EXPERTS);
+      const int max_smem = (int)L::bytes(GG_MAX_EXPERTS);
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) !=
           cudaSuccess)
         return GG_ERR_CUDA;
+      int units = di.sms;
+      if (PAIR) {
+        // persistent grid: as many CTA pairs as can be resident at once
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3(2 * (di.sms / 2), 1, 1);
+        cfg.blockDim = dim3(gg::NUM_THREADS, 1, 1);
+        cfg.dynamicSmemBytes = (size_t)max_smem;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1)
+          return GG_ERR_CUDA;
+        units = clusters;
+      }
+      max_units[dev] = units;
       attr_done[dev] = true;
     }
   }
-  int64_t grid = tiles_upper < di.sms ? tiles_upper : di.sms;
-  if (grid < 1) grid = 1;
-  kern<<<(unsigned)grid, gg::NUM_THREADS, smem, stream>>>(a, b, p);
+  int64_t units = tiles_upper < max_units[dev] ? tiles_upper : max_units[dev];
+  if (units < 1) units = 1;
+  if (!PAIR) {
+    kern<<<(unsigned)units, gg::NUM_THREADS, smem, stream>>>(a, b, p);
+    return cudaGetLastError() == cudaSuccess ? GG_OK : GG_ERR_CUDA;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3((unsigned)(2 * units), 1, 1);
+  cfg.blockDim = dim3(gg::NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, a, b, p) != cudaSuccess) return GG_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? GG_OK : GG_ERR_CUDA;
 }
 
@@ -172,7 +211,17 @@ gg_status check_common(int64_t rows_alloc, int64_t K, int64_t N, int32_t E,
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 constexpr int kBN = 256;
-constexpr int kStages = 4;
+constexpr int kStages = 4;      // single CTA: 48 KB per stage
+constexpr int kPairStages = 6;  // CTA pair: 32 KB per stage and CTA
+
+// CTA pairs halve the operand traffic per SM but quantise groups to 256-row tiles; they pay
+// off once the average group is long.
+bool use_pair(int64_t rows, int32_t E) {
+  const int v = g_force_variant.load();
+  if (v == 1) return false;
+  if (v == 2) return true;
+  return rows >= 512 * (int64_t)E;
+}
 
 }  // namespace
 
@@ -194,8 +243,12 @@ gg_status gg_forward(const void* A, const void* W, const int32_t* offs, void* ou
   gg::Params p = base_params(offs, out, dev_status, rows_alloc, E);
   p.red_len = (int32_t)K;
   p.out_cols = (int32_t)N;
+  if (use_pair(rows_alloc, E)) {
+    const int64_t tiles = (cdiv(rows_alloc, 2 * gg::BM) + E) * cdiv(N, kBN);
+    return launch<Mode::Forward, kBN, kPairStages, true>(ma, mb, p, tiles, di, stream);
+  }
   const int64_t tiles = (cdiv(rows_alloc, gg::BM) + E) * cdiv(N, kBN);
-  return launch<Mode::Forward, kBN, kStages>(ma, mb, p, tiles, di, stream);
+  return launch<Mode::Forward, kBN, kStages, false>(ma, mb, p, tiles, di, stream);
 }
 
 gg_status gg_dgrad(const void* dY, const void* W, const int32_t* offs, void* dX,
@@ -209,13 +262,19 @@ gg_status gg_dgrad(const void* dY, const void* W, const int32_t* offs, void* dX,
   if (dY == nullptr || dX == nullptr) return GG_ERR_INVALID_ARG;
   if (!aligned16(dY) || !aligned16(W) || !aligned16(dX)) return GG_ERR_UNSUPPORTED;
   CUtensorMap ma, mb;
-  if (!map_2d(&ma, dY, rows_alloc, N, 64, gg::BM) || !map_w(&mb, W, E, K, N, 64, kBN))
+  const bool pair = use_pair(rows_alloc, E);
+  if (!map_2d(&ma, dY, rows_alloc, N, 64, gg::BM) ||
+      !map_w(&mb, W, E, K, N, 64, pair ? kBN / 2 : kBN))
     return GG_ERR_CUDA;
   gg::Params p = base_params(offs, dX, dev_status, rows_alloc, E);
   p.red_len = (int32_t)N;
   p.out_cols = (int32_t)K;
+  if (pair) {
+    const int64_t tiles = (cdiv(rows_alloc, 2 * gg::BM) + E) * cdiv(K, kBN);
+    return launch<Mode::Dgrad, kBN, kPairStages, true>(ma, mb, p, tiles, di, stream);
+  }
   const int64_t tiles = (cdiv(rows_alloc, gg::BM) + E) * cdiv(K, kBN);
-  return launch<Mode::Dgrad, kBN, kStages>(ma, mb, p, tiles, di, stream);
+  return launch<Mode::Dgrad, kBN, kStages, false>(ma, mb, p, tiles, di, stream);
 }
 
 gg_status gg_wgrad(const void* A, const void* dY, const int32_t* offs, void* dW,
@@ -241,7 +300,7 @@ gg_status gg_wgrad(const void* A, const void* dY, const int32_t* offs, void* dW,
   p.out_cols = (int32_t)N;
   p.wg_K = (int32_t)K;
   const int64_t tiles = (int64_t)E * cdiv(K, gg::BM) * cdiv(N, kBN);
-  return launch<Mode::Wgrad, kBN, kStages>(ma, mb, p, tiles, di, stream);
+  return launch<Mode::Wgrad, kBN, kStages, false>(ma, mb, p, tiles, di, stream);
 }
 
 gg_status gg_masked_forward(const void* A, const void* W, const int32_t* masked_m, void* out,
@@ -264,7 +323,7 @@ gg_status gg_masked_forward(const void* A, const void* W, const int32_t* masked_
   p.red_len = (int32_t)K;
   p.out_cols = (int32_t)N;
   const int64_t tiles = (int64_t)E * cdiv(mmax, gg::BM) * cdiv(N, kBN);
-  return launch<Mode::Masked, kBN, kStages>(ma, mb, p, tiles, di, stream);
+  return launch<Mode::Masked, kBN, kStages, false>(ma, mb, p, tiles, di, stream);
 }
 
 const char* gg_status_string(gg_status s) {
@@ -283,6 +342,10 @@ uint64_t gg_set_watchdog_ns(uint64_t ns) {
 }
 
 int gg_testing_skip_first_load(int enable) { return g_skip_first_load.exchange(enable ? 1 : 0); }
+
+int gg_testing_force_variant(int variant) {
+  return g_force_variant.exchange(variant == 1 || variant == 2 ? variant : 0);
+}
 
 int gg_version(void) { return 100; }
 

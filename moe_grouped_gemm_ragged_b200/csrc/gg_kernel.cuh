@@ -7,6 +7,13 @@
 //   Wgrad    dW[e]      = A[rows of e]^T . dY[rows of e] (tile rows = K index; the reduction
 //                                                        runs over the ragged token rows)
 //
+// Two launch shapes share this code:
+//   single CTA (PAIR = false): a tile is 128 rows x BN columns, one CTA per SM;
+//   CTA pair   (PAIR = true):  a cluster of 2 CTAs on neighbouring SMs computes one
+//               256 x BN tile with tcgen05.mma.cta_group::2: each CTA loads its own 128 rows
+//               of A and its own BN/2 columns of B (no multicast), the pair leader issues the
+//               MMAs, and each CTA's tensor memory holds its 128 rows of the accumulator.
+//
 // Roles of the 6 warps of a CTA (one CTA per SM, persistent over a strided tile list):
 //   warp 0      TMA producer: one lane arms a stage barrier and issues the tensor loads
 //   warp 1      tensor-memory owner and MMA issuer: one lane issues tcgen05.mma into a
@@ -58,10 +65,11 @@ struct Params {
   int32_t debug_flags;     // bit 0: CTA 0 skips its first load (watchdog test)
 };
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool PAIR>
 struct Layout {
+  static constexpr int B_COLS = PAIR ? BN / 2 : BN;  // columns of B this CTA loads
   static constexpr uint32_t A_BYTES = BM * BK * 2;
-  static constexpr uint32_t B_BYTES = BN * BK * 2;
+  static constexpr uint32_t B_BYTES = B_COLS * BK * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr uint32_t OFF_A = 0;
   static constexpr uint32_t OFF_B = STAGES * A_BYTES;
@@ -108,13 +116,18 @@ __device__ __forceinline__ void set_status(const Params& p, int bits) {
 }
 
 // Bounded wait on one phase of an mbarrier. Returns false when the CTA is aborting or the
-// watchdog expired (then the abort flag and GG_DEV_TIMEOUT are set).
+// watchdog expired (then the abort flag and GG_DEV_TIMEOUT are set). `cluster` selects
+// acquire at cluster scope, for barriers that receive arrivals from the peer CTA.
 __device__ __noinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, const Shared& sh,
-                                          const Params& p, bool honour_abort) {
-  if (ptx::mbar_try_wait(bar, parity)) return true;
+                                          const Params& p, bool honour_abort,
+                                          bool cluster = false) {
+  auto probe = [&]() {
+    return cluster ? ptx::mbar_try_wait_cluster(bar, parity) : ptx::mbar_try_wait(bar, parity);
+  };
+  if (probe()) return true;
   const uint64_t t0 = ptx::globaltimer();
   for (uint32_t i = 1;; ++i) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (probe()) return true;
     if ((i & 31u) == 0u) {
       if (honour_abort && *sh.abort_flag) return false;
       if (ptx::globaltimer() - t0 > p.watchdog_ns) {
@@ -128,9 +141,9 @@ __device__ __noinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, const 
 
 // Single-lane wait whose outcome every lane of the warp shares.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const Shared& sh,
-                                          const Params& p) {
+                                          const Params& p, bool cluster) {
   bool ok = true;
-  if (ptx::lane_id() == 0) ok = wait_bounded(bar, parity, sh, p, true);
+  if (ptx::lane_id() == 0) ok = wait_bounded(bar, parity, sh, p, true, cluster);
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
@@ -138,7 +151,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
 // Warp 0 builds the group table. Ragged modes: effective ends t'_e = clamp(offs[e],
 // t'_{e-1}, rows_alloc) with t'_{-1} = 0, i.e. min(running max of offs (from 0), rows).
 // Masked: group e starts at e*mmax and has clamp(masked_m[e], 0, mmax) rows.
-template <Mode MODE, int BN>
+template <Mode MODE, int BN, int TM>
 __device__ void build_table(const Params& p, const Shared& sh) {
   const uint32_t lane = ptx::lane_id();
   const int32_t E = p.E;
@@ -180,7 +193,7 @@ __device__ void build_table(const Params& p, const Shared& sh) {
       if constexpr (MODE == Mode::Wgrad) {
         tiles = 0;  // fixed grid, counted below
       } else {
-        tiles = ((end - start + BM - 1) / BM) * NT;
+        tiles = ((end - start + TM - 1) / TM) * NT;
       }
     }
     int32_t s = tiles;
@@ -223,7 +236,7 @@ __device__ void build_wgrad_order(const Params& p, const Shared& sh) {
   }
 }
 
-template <Mode MODE, int BN>
+template <Mode MODE, int BN, int TM>
 __device__ __forceinline__ Tile decode_tile(int32_t t, const Params& p, const Shared& sh) {
   Tile tl;
   const int32_t NT = (p.out_cols + BN - 1) / BN;
@@ -256,7 +269,7 @@ __device__ __forceinline__ Tile decode_tile(int32_t t, const Params& p, const Sh
     const int32_t mt = local / NT;
     const int32_t nt = local - mt * NT;
     tl.e = e;
-    tl.a_row0 = sh.gstart[e] + mt * BM;
+    tl.a_row0 = sh.gstart[e] + mt * TM;
     tl.row0 = tl.a_row0;
     tl.row_end = sh.gend[e];
     tl.n0 = nt * BN;
@@ -269,18 +282,22 @@ __device__ __forceinline__ Tile decode_tile(int32_t t, const Params& p, const Sh
 }
 
 // ---------------------------------------------------------------- kernel
-template <Mode MODE, int BN, int STAGES>
+template <Mode MODE, int BN, int STAGES, bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap mapA,
                         const __grid_constant__ CUtensorMap mapB, const Params p) {
-  using L = Layout<BN, STAGES>;
+  using L = Layout<BN, STAGES, PAIR>;
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN must be 64, 128, 192 or 256");
+  static_assert(!PAIR || BN % 128 == 0, "a CTA pair splits BN into two multiples of 64");
+  static_assert(!(PAIR && MODE == Mode::Wgrad), "wgrad runs on single CTAs");
   static_assert(L::TMEM_COLS == 128 || L::TMEM_COLS == 256 || L::TMEM_COLS == 512,
                 "TMEM allocation must be a power of two");
+  constexpr int TM = PAIR ? 2 * BM : BM;  // rows of a tile
   // A operand MN-major only in Wgrad; B operand K-major only in Dgrad.
   constexpr uint32_t A_MN = (MODE == Mode::Wgrad) ? 1u : 0u;
   constexpr uint32_t B_MN = (MODE == Mode::Dgrad) ? 0u : 1u;
-  constexpr uint32_t IDESC = ptx::idesc_bf16_f32(BM, BN, A_MN, B_MN);
+  constexpr uint32_t IDESC = ptx::idesc_bf16_f32(TM, BN, A_MN, B_MN);
+  constexpr uint32_t EPI_ARRIVALS = PAIR ? 8u : 4u;  // one per epilogue warp of the tile
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = ptx::smem_u32(smem_raw);
@@ -304,6 +321,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const uint32_t warp = threadIdx.x / 32;
   const uint32_t lane = ptx::lane_id();
+  const uint32_t rank = PAIR ? ptx::cluster_ctarank() : 0u;  // 0 = pair leader
+  const bool leader = rank == 0;
+  const int32_t unit0 = PAIR ? (int32_t)ptx::cluster_id_x() : (int32_t)blockIdx.x;
+  const int32_t units = PAIR ? (int32_t)ptx::ncluster_x() : (int32_t)gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -312,7 +333,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       ptx::mbar_init(&sh.tfull[a], 1);
-      ptx::mbar_init(&sh.tempty[a], 128);
+      ptx::mbar_init(&sh.tempty[a], EPI_ARRIVALS);
     }
     ptx::mbar_init(sh.fin, 1);
     *sh.abort_flag = 0;
@@ -321,12 +342,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::prefetch_tmap(&mapB);
   }
   if (warp == 1) {
-    ptx::tmem_alloc(sh.tmem_base, L::TMEM_COLS);
-    ptx::tmem_relinquish();
+    if constexpr (PAIR) {
+      ptx::tmem_alloc_pair(sh.tmem_base, L::TMEM_COLS);
+      ptx::tmem_relinquish_pair();
+    } else {
+      ptx::tmem_alloc(sh.tmem_base, L::TMEM_COLS);
+      ptx::tmem_relinquish();
+    }
   }
-  if (warp == 0) build_table<MODE, BN>(p, sh);
+  if (warp == 0) build_table<MODE, BN, TM>(p, sh);
   ptx::tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) ptx::cluster_sync();  // peer barriers initialised before any remote use
+  else __syncthreads();
   ptx::tc_fence_after();
   if constexpr (MODE == Mode::Wgrad) {
     build_wgrad_order(p, sh);
@@ -344,8 +371,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t armed = 0, armed_par = 0;  // per-stage: loads in flight, and their phase
       bool skip_first = (p.debug_flags & 1) && blockIdx.x == 0;
       bool ok = true;
-      for (int32_t t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const Tile tl = decode_tile<MODE, BN>(t, p, sh);
+      const int32_t row_off = (int32_t)rank * BM;       // this CTA's rows of a pair tile
+      const int32_t col_off = (int32_t)rank * L::B_COLS;  // this CTA's columns of B
+      for (int32_t t = unit0; t < total && ok; t += units) {
+        const Tile tl = decode_tile<MODE, BN, TM>(t, p, sh);
         for (int32_t kb = 0; kb < tl.kblocks; ++kb) {
           if (!wait_bounded(&sh.empty[stage], phase ^ 1u, sh, p, true)) { ok = false; break; }
           armed &= ~(1u << stage);
@@ -354,6 +383,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint64_t* fb = &sh.full[stage];
           if (skip_first) {
             skip_first = false;  // watchdog test: never arm this stage
+          } else if constexpr (PAIR) {
+            // the leader's full barrier counts the bytes of both CTAs
+            const uint32_t fb_leader = ptx::mapa(ptx::smem_u32(fb), 0);
+            if (leader) ptx::mbar_arrive_expect_tx(fb, 2 * L::STAGE_BYTES);
+            ptx::tma_load_2d_pair(sA, &mapA, fb_leader, kb * BK, tl.a_row0 + row_off,
+                                  pol_stream);
+            if constexpr (MODE == Mode::Dgrad) {
+              ptx::tma_load_3d_pair(sB, &mapB, fb_leader, kb * BK, tl.n0 + col_off, tl.e,
+                                    pol_keep);
+            } else {
+#pragma unroll
+              for (int j = 0; j < L::B_COLS / 64; ++j)
+                ptx::tma_load_3d_pair(sB + j * 8192, &mapB, fb_leader, tl.n0 + col_off + j * 64,
+                                      kb * BK, tl.e, pol_keep);
+            }
+            if (leader) {
+              armed |= 1u << stage;
+              armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+            }
           } else {
             ptx::mbar_arrive_expect_tx(fb, L::STAGE_BYTES);
             if constexpr (MODE == Mode::Forward || MODE == Mode::Masked) {
@@ -380,88 +428,119 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
-      // Let every load this thread issued land before the CTA can exit (on the normal path
+      // Let every load this thread armed land before the CTA can exit (on the normal path
       // these phases have completed already; after an abort some may still be in flight).
+      // A pair follower's loads complete on the leader's barriers; they were issued at least
+      // one watchdog period before any abort could end this CTA.
       for (int s = 0; s < STAGES; ++s)
         if (armed & (1u << s)) wait_bounded(&sh.full[s], (armed_par >> s) & 1u, sh, p, false);
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    uint32_t stage = 0, phase = 0, acc_iter = 0;
-    bool ok = true;
-    for (int32_t t = blockIdx.x; t < total && ok; t += gridDim.x) {
-      const Tile tl = decode_tile<MODE, BN>(t, p, sh);
-      if (tl.kblocks == 0) continue;  // Wgrad of an empty expert: the epilogue writes zeros
-      const uint32_t a = acc_iter & 1u;
-      if (!warp_wait(&sh.tempty[a], ((acc_iter >> 1) & 1u) ^ 1u, sh, p)) { ok = false; break; }
-      ptx::tc_fence_after();
-      const uint32_t d_tmem = tmem_base + a * BN;
-      for (int32_t kb = 0; kb < tl.kblocks; ++kb) {
-        if (!warp_wait(&sh.full[stage], phase, sh, p)) { ok = false; break; }
-        ptx::tc_fence_after();
-        uint8_t* sA = smem + L::OFF_A + stage * L::A_BYTES;
-        uint8_t* sB = smem + L::OFF_B + stage * L::B_BYTES;
-        int nsub = BK / UMMA_K;
-        if constexpr (MODE == Mode::Wgrad) {
-          const int32_t rem = tl.tok_len - kb * BK;  // rows of this group in the stage
-          if (rem < BK) {
-            nsub = (rem + UMMA_K - 1) / UMMA_K;
-            // Rows [rem, nsub*16) belong to the next group (or to no group): zero them in
-            // both operands so they add nothing. Each token row is one 128-byte line of
-            // every 64-wide chunk.
-            const int zrows = nsub * UMMA_K - rem;
-            const int lines_a = zrows * 2, lines_b = zrows * (BN / 64);
-            for (int i = (int)lane; i < (lines_a + lines_b) * 8; i += 32) {
-              const int line = i >> 3, part = i & 7;
-              uint8_t* dst;
-              if (line < lines_a) {
-                const int c = line / zrows, rr = rem + line % zrows;
-                dst = sA + c * 8192 + rr * 128 + part * 16;
-              } else {
-                const int l2 = line - lines_a;
-                const int c = l2 / zrows, rr = rem + l2 % zrows;
-                dst = sB + c * 8192 + rr * 128 + part * 16;
-              }
-              *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
-            }
-            ptx::fence_proxy_async_smem();
-            __syncwarp();
-          }
+    // ------------------------------------------------------------ MMA issuer (pair leader)
+    if (leader) {
+      uint32_t stage = 0, phase = 0, acc_iter = 0;
+      bool ok = true;
+      for (int32_t t = unit0; t < total && ok; t += units) {
+        const Tile tl = decode_tile<MODE, BN, TM>(t, p, sh);
+        if (tl.kblocks == 0) continue;  // Wgrad of an empty expert: the epilogue writes zeros
+        const uint32_t a = acc_iter & 1u;
+        if (!warp_wait(&sh.tempty[a], ((acc_iter >> 1) & 1u) ^ 1u, sh, p, PAIR)) {
+          ok = false;
+          break;
         }
-        if (lane == 0) {
-          const uint32_t a_base = ptx::smem_u32(sA), b_base = ptx::smem_u32(sB);
-          for (int k = 0; k < nsub; ++k) {
-            uint64_t adesc, bdesc;
-            if constexpr (A_MN) adesc = ptx::smem_desc_sw128(a_base + k * 2048, 8192, 1024);
-            else                adesc = ptx::smem_desc_sw128(a_base + k * 32, 16, 1024);
-            if constexpr (B_MN) bdesc = ptx::smem_desc_sw128(b_base + k * 2048, 8192, 1024);
-            else                bdesc = ptx::smem_desc_sw128(b_base + k * 32, 16, 1024);
-            ptx::mma_bf16(d_tmem, adesc, bdesc, IDESC, (kb > 0 || k > 0) ? 1u : 0u);
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + a * BN;
+        for (int32_t kb = 0; kb < tl.kblocks; ++kb) {
+          if (!warp_wait(&sh.full[stage], phase, sh, p, false)) { ok = false; break; }
+          ptx::tc_fence_after();
+          uint8_t* sA = smem + L::OFF_A + stage * L::A_BYTES;
+          uint8_t* sB = smem + L::OFF_B + stage * L::B_BYTES;
+          int nsub = BK / UMMA_K;
+          if constexpr (MODE == Mode::Wgrad) {
+            const int32_t rem = tl.tok_len - kb * BK;  // rows of this group in the stage
+            if (rem < BK) {
+              nsub = (rem + UMMA_K - 1) / UMMA_K;
+              // Rows [rem, nsub*16) belong to the next group (or to no group): zero them in
+              // both operands so they add nothing. Each token row is one 128-byte line of
+              // every 64-wide chunk.
+              const int zrows = nsub * UMMA_K - rem;
+              const int lines_a = zrows * 2, lines_b = zrows * (BN / 64);
+              for (int i = (int)lane; i < (lines_a + lines_b) * 8; i += 32) {
+                const int line = i >> 3, part = i & 7;
+                uint8_t* dst;
+                if (line < lines_a) {
+                  const int c = line / zrows, rr = rem + line % zrows;
+                  dst = sA + c * 8192 + rr * 128 + part * 16;
+                } else {
+                  const int l2 = line - lines_a;
+                  const int c = l2 / zrows, rr = rem + l2 % zrows;
+                  dst = sB + c * 8192 + rr * 128 + part * 16;
+                }
+                *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+              }
+              ptx::fence_proxy_async_smem();
+              __syncwarp();
+            }
           }
-          ptx::mma_commit(&sh.empty[stage]);  // frees the stage once these MMAs are done
+          if (lane == 0) {
+            const uint32_t a_base = ptx::smem_u32(sA), b_base = ptx::smem_u32(sB);
+            for (int k = 0; k < nsub; ++k) {
+              uint64_t adesc, bdesc;
+              if constexpr (A_MN) adesc = ptx::smem_desc_sw128(a_base + k * 2048, 8192, 1024);
+              else                adesc = ptx::smem_desc_sw128(a_base + k * 32, 16, 1024);
+              if constexpr (B_MN) bdesc = ptx::smem_desc_sw128(b_base + k * 2048, 8192, 1024);
+              else                bdesc = ptx::smem_desc_sw128(b_base + k * 32, 16, 1024);
+              const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+              if constexpr (PAIR) ptx::mma_bf16_pair(d_tmem, adesc, bdesc, IDESC, acc);
+              else                ptx::mma_bf16(d_tmem, adesc, bdesc, IDESC, acc);
+            }
+            // free the stage (in both CTAs of a pair) once these MMAs are done
+            if constexpr (PAIR) {
+              const uint32_t eb = ptx::smem_u32(&sh.empty[stage]);
+              ptx::mma_commit_pair(ptx::mapa(eb, 0));
+              ptx::mma_commit_pair(ptx::mapa(eb, 1));
+            } else {
+              ptx::mma_commit(&sh.empty[stage]);
+            }
+          }
+          __syncwarp();
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        if (lane == 0) {
+          if constexpr (PAIR) {
+            const uint32_t fb = ptx::smem_u32(&sh.tfull[a]);
+            ptx::mma_commit_pair(ptx::mapa(fb, 0));
+            ptx::mma_commit_pair(ptx::mapa(fb, 1));
+          } else {
+            ptx::mma_commit(&sh.tfull[a]);
+          }
         }
         __syncwarp();
-        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        ++acc_iter;
       }
-      if (!ok) break;
-      if (lane == 0) ptx::mma_commit(&sh.tfull[a]);
+      // every MMA issued by this CTA completes before tensor memory is released
+      if (lane == 0) {
+        if constexpr (PAIR) ptx::mma_commit_pair(ptx::mapa(ptx::smem_u32(sh.fin), 0));
+        else                ptx::mma_commit(sh.fin);
+        wait_bounded(sh.fin, 0, sh, p, false);
+      }
       __syncwarp();
-      ++acc_iter;
     }
-    // every MMA issued by this CTA completes before tensor memory is released
-    if (lane == 0) {
-      ptx::mma_commit(sh.fin);
-      wait_bounded(sh.fin, 0, sh, p, false);
-    }
-    __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
     const uint32_t q = warp & 3u;  // TMEM lane quadrant this warp may access
-    const int32_t row_in_tile = (int32_t)(q * 32 + lane);
+    const int32_t row_in_tile = (int32_t)(rank * BM + q * 32 + lane);
+    // tensor memory of this CTA's accumulator is released on the pair leader's barrier
+    uint32_t tempty0 = ptx::smem_u32(&sh.tempty[0]), tempty1 = ptx::smem_u32(&sh.tempty[1]);
+    if constexpr (PAIR) {
+      tempty0 = ptx::mapa(tempty0, 0);
+      tempty1 = ptx::mapa(tempty1, 0);
+    }
     uint32_t acc_iter = 0;
-    for (int32_t t = blockIdx.x; t < total; t += gridDim.x) {
-      const Tile tl = decode_tile<MODE, BN>(t, p, sh);
+    for (int32_t t = unit0; t < total; t += units) {
+      const Tile tl = decode_tile<MODE, BN, TM>(t, p, sh);
       const int64_t orow = tl.row0 + row_in_tile;
       const bool row_ok = orow < tl.row_end;
       __nv_bfloat16* orow_ptr = p.out + orow * (int64_t)p.out_cols;
@@ -476,7 +555,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         continue;
       }
       const uint32_t a = acc_iter & 1u;
-      if (!warp_wait(&sh.tfull[a], (acc_iter >> 1) & 1u, sh, p)) break;
+      if (!warp_wait(&sh.tfull[a], (acc_iter >> 1) & 1u, sh, p, false)) break;
       ptx::tc_fence_after();
       const uint32_t taddr = tmem_base + ((q * 32u) << 16) + a * BN;
 #pragma unroll 1
@@ -503,16 +582,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       ptx::tc_fence_before();
-      ptx::mbar_arrive(&sh.tempty[a]);
+      __syncwarp();
+      if (lane == 0) {
+        if constexpr (PAIR) ptx::mbar_arrive_cluster(a ? tempty1 : tempty0);
+        else                ptx::mbar_arrive(&sh.tempty[a]);
+      }
       ++acc_iter;
     }
   }
 
   ptx::tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) ptx::cluster_sync();  // no CTA of the pair leaves while the other may
+  else __syncthreads();                      // still signal its barriers or tensor memory
   if (warp == 1) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem_base, L::TMEM_COLS);
+    if constexpr (PAIR) ptx::tmem_dealloc_pair(tmem_base, L::TMEM_COLS);
+    else                ptx::tmem_dealloc(tmem_base, L::TMEM_COLS);
   }
   if (blockIdx.x == 0 && threadIdx.x == 0 && !*sh.abort_flag) set_status(p, DEV_LAUNCHED);
 }

@@ -19,6 +19,14 @@ pytestmark = [pytest.mark.gpu,
 gg = pytest.importorskip("moe_grouped_gemm_ragged_b200")
 
 
+@pytest.fixture(params=[1, 2], ids=["single_cta", "cta_pair"])
+def variant(request):
+    """Run forward/dgrad with 128-row single-CTA tiles and with 256-row CTA-pair tiles."""
+    prev = gg.testing_force_variant(request.param)
+    yield request.param
+    gg.testing_force_variant(prev)
+
+
 def _dev(r: workloads.RaggedInputs):
     return (r.A.cuda(), r.W.cuda(), r.dY.cuda(),
             torch.from_numpy(np.ascontiguousarray(r.offs)).cuda())
@@ -74,7 +82,7 @@ def check_ragged(r: workloads.RaggedInputs, sample: bool, seed: int = 0,
 @pytest.mark.parametrize("offs", [(8, 16, 32, 40), (8, 8, 32, 40), (0, 16, 32, 40),
                                   (8, 16, 32, 32), (0, 0, 0, 0), (40, 40, 40, 40),
                                   (48, 48, 48, 48), (0, 0, 0, 48)])
-def test_tiny_repro_offsets(offs):
+def test_tiny_repro_offsets(offs, variant):
     """The 4-expert M=48/K=8/N=16 repro with its two offset tuples and edge variants."""
     r = workloads.make_tiny(offs)
     out, dX, dW = check_ragged(r, sample=False)
@@ -86,20 +94,20 @@ SWEEP = [0, 1, 7, 8, 9, 15, 16, 17, 127, 128, 129, 255, 256, 257]
 
 
 @pytest.mark.parametrize("K,N", [(200, 328), (64, 256), (8, 16), (136, 520)])
-def test_group_size_sweep(K, N):
+def test_group_size_sweep(K, N, variant):
     """Group sizes around 0, 8, 16, 128 and 256 rows, K and N tails, NaN tail rows."""
     r = workloads.make_ragged_custom(len(SWEEP), K, N, SWEEP, seed=100 + K, tail=128)
     check_ragged(r, sample=False)
 
 
-def test_shuffled_sizes_many_experts():
+def test_shuffled_sizes_many_experts(variant):
     rng = np.random.default_rng(7)
     sizes = rng.permutation(np.array(SWEEP * 3))
     r = workloads.make_ragged_custom(len(sizes), 256, 384, sizes, seed=8, tail=200)
     check_ragged(r, sample=False)
 
 
-def test_group_id_probe_bit_exact():
+def test_group_id_probe_bit_exact(variant):
     """A[:,0]=1, W[e][0,:]=e+1: every output row equals its group id + 1 exactly."""
     sizes = [3, 0, 130, 1, 257, 0, 64]
     E, K, N = len(sizes), 64, 264
@@ -140,7 +148,7 @@ def test_masked_config_full():
 
 
 @pytest.mark.parametrize("name", ["gateup", "downproj"])
-def test_moe_projection_configs(name):
+def test_moe_projection_configs(name, variant):
     """E=64 Zipf gate-up (K=2048, N=1536) and E=32 down-proj (K=2048, N=7168): sampled rows
     {s, s+1, t-2, t-1} + 60 random per group and 32 K rows per expert, NaN tail rows."""
     r = workloads.make_ragged(name, tail=128, device="cuda")
@@ -149,13 +157,13 @@ def test_moe_projection_configs(name):
 
 @pytest.mark.slow
 @pytest.mark.parametrize("name", ["large", "large_unaligned"])
-def test_large_configs(name):
+def test_large_configs(name, variant):
     """262144 x 6144 x 4096, E=16, aligned and +-1..127 perturbed sizes (sampled)."""
     r = workloads.make_ragged(name, tail=128, device="cuda")
     check_ragged(r, sample=True, seed=2)
 
 
-def test_repeat_calls_bit_identical():
+def test_repeat_calls_bit_identical(variant):
     r = workloads.make_ragged_custom(5, 192, 512, [100, 0, 300, 7, 513], seed=3, tail=9)
     a = run_ragged(r)
     b = run_ragged(r)
