@@ -392,7 +392,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="large",
-                    choices=["large", "large_unaligned", "gateup", "downproj"])
+                    choices=["large", "large_unaligned", "gateup", "downproj", "large_e2"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")

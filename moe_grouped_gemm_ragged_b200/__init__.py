@@ -18,7 +18,8 @@ from typing import Optional
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libgg.so")
+# GG_LIBRARY may name another build of the same library (e.g. with other tuning macros)
+LIB_PATH = os.environ.get("GG_LIBRARY") or os.path.join(_PKG, "libgg.so")
 
 GG_OK, GG_ERR_INVALID_ARG, GG_ERR_UNSUPPORTED, GG_ERR_CUDA = 0, 1, 2, 3
 DEV_BAD_OFFSETS = 0x1

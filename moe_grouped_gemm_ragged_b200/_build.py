@@ -46,18 +46,23 @@ def stale() -> bool:
     return any(os.path.getmtime(f) > t for f in _inputs())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile ``csrc/*.cu`` into ``libgg.so`` (sm_100a) unless it is up to date."""
-    if not force and not stale():
+def build(force: bool = False, verbose: bool = False, out: str = None, defines=()) -> str:
+    """Compile ``csrc/*.cu`` into ``libgg.so`` (sm_100a) unless it is up to date.
+
+    ``out`` and ``defines`` (``NAME=VALUE`` strings) build another copy with other tuning
+    macros; such a copy is always rebuilt."""
+    target = out or LIB
+    if out is None and not force and not stale():
         return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, *sources(), "-o", tmp]
+    tmp = target + f".tmp{os.getpid()}"
+    cmd = [_nvcc(), *NVCC_FLAGS, *[f"-D{d}" for d in defines], "-I", INCLUDE, "-I", CSRC,
+           *sources(), "-o", tmp]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), file=sys.stderr)
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, target)
+    return target
 
 
 if __name__ == "__main__":

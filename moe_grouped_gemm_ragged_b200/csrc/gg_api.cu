@@ -80,10 +80,10 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
               const uint64_t* strides_bytes, const uint32_t* box) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
-  cuuint64_t gdim[3];
-  cuuint64_t gstr[2];
-  cuuint32_t bdim[3];
-  cuuint32_t estr[3] = {1, 1, 1};
+  cuuint64_t gdim[4];
+  cuuint64_t gstr[3];
+  cuuint32_t bdim[4];
+  cuuint32_t estr[4] = {1, 1, 1, 1};
   for (int i = 0; i < rank; ++i) {
     gdim[i] = dims[i];
     bdim[i] = box[i];
@@ -104,6 +104,28 @@ bool map_2d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32
   const uint64_t str[1] = {(uint64_t)cols * 2u};
   const uint32_t box[2] = {box_cols, box_rows};
   return make_map(m, base, 2, dims, str, box);
+}
+
+// 3-D map over a row-major [rows, cols] bf16 matrix whose columns are split into 64-wide
+// chunks (dims innermost first: 64, rows, cols/64): one box of `nchunks` chunks x box_rows
+// rows lands in shared memory as [chunk][row][64]. Needs cols % 64 == 0.
+bool map_2d_chunked(CUtensorMap* m, const void* base, int64_t rows, int64_t cols,
+                    uint32_t box_rows, uint32_t nchunks) {
+  const uint64_t dims[3] = {64u, (uint64_t)(rows > 0 ? rows : 1), (uint64_t)cols / 64u};
+  const uint64_t str[2] = {(uint64_t)cols * 2u, 128u};
+  const uint32_t box[3] = {64u, box_rows, nchunks};
+  return make_map(m, base, 3, dims, str, box);
+}
+
+// 4-D map over W[E, K, N] with N split into 64-wide chunks (dims innermost first: 64, K,
+// N/64, E): one box of `nchunks` chunks x box_k rows of K lands as [chunk][k][64].
+// Needs N % 64 == 0.
+bool map_w_chunked(CUtensorMap* m, const void* W, int64_t E, int64_t K, int64_t N,
+                   uint32_t box_k, uint32_t nchunks) {
+  const uint64_t dims[4] = {64u, (uint64_t)K, (uint64_t)N / 64u, (uint64_t)E};
+  const uint64_t str[3] = {(uint64_t)N * 2u, 128u, (uint64_t)K * (uint64_t)N * 2u};
+  const uint32_t box[4] = {64u, box_k, nchunks, 1u};
+  return make_map(m, W, 4, dims, str, box);
 }
 
 // 3-D map over the packed weights W[E, K, N] (dims innermost first: N, K, E).
@@ -237,13 +259,18 @@ gg_status gg_forward(const void* A, const void* W, const int32_t* offs, void* ou
   if (rows_alloc == 0) return GG_OK;  // no row can belong to a group
   if (A == nullptr || out == nullptr) return GG_ERR_INVALID_ARG;
   if (!aligned16(A) || !aligned16(W) || !aligned16(out)) return GG_ERR_UNSUPPORTED;
+  const bool pair = use_pair(rows_alloc, E);
+  const bool chunked = (N % 64) == 0;
+  const uint32_t bcols = pair ? kBN / 2 : kBN;
   CUtensorMap ma, mb;
-  if (!map_2d(&ma, A, rows_alloc, K, 64, gg::BM) || !map_w(&mb, W, E, K, N, 64, 64))
+  if (!map_2d(&ma, A, rows_alloc, K, 64, gg::BM)) return GG_ERR_CUDA;
+  if (chunked ? !map_w_chunked(&mb, W, E, K, N, 64, bcols / 64) : !map_w(&mb, W, E, K, N, 64, 64))
     return GG_ERR_CUDA;
   gg::Params p = base_params(offs, out, dev_status, rows_alloc, E);
   p.red_len = (int32_t)K;
   p.out_cols = (int32_t)N;
-  if (use_pair(rows_alloc, E)) {
+  p.b_chunked = chunked ? 1 : 0;
+  if (pair) {
     const int64_t tiles = (cdiv(rows_alloc, 2 * gg::BM) + E) * cdiv(N, kBN);
     return launch<Mode::Forward, kBN, kPairStages, true>(ma, mb, p, tiles, di, stream);
   }
@@ -293,12 +320,19 @@ gg_status gg_wgrad(const void* A, const void* dY, const int32_t* offs, void* dW,
     A = dW;
     dY = dW;
   }
+  const bool a_chunked = (K % 64) == 0, b_chunked = (N % 64) == 0;
   CUtensorMap ma, mb;
-  if (!map_2d(&ma, A, rows_alloc, K, 64, 64) || !map_2d(&mb, dY, rows_alloc, N, 64, 64))
+  if (a_chunked ? !map_2d_chunked(&ma, A, rows_alloc, K, 64, gg::BM / 64)
+                : !map_2d(&ma, A, rows_alloc, K, 64, 64))
+    return GG_ERR_CUDA;
+  if (b_chunked ? !map_2d_chunked(&mb, dY, rows_alloc, N, 64, kBN / 64)
+                : !map_2d(&mb, dY, rows_alloc, N, 64, 64))
     return GG_ERR_CUDA;
   gg::Params p = base_params(offs, dW, dev_status, rows_alloc, E);
   p.out_cols = (int32_t)N;
   p.wg_K = (int32_t)K;
+  p.a_chunked = a_chunked ? 1 : 0;
+  p.b_chunked = b_chunked ? 1 : 0;
   const int64_t tiles = (int64_t)E * cdiv(K, gg::BM) * cdiv(N, kBN);
   return launch<Mode::Wgrad, kBN, kStages, false>(ma, mb, p, tiles, di, stream);
 }
@@ -315,10 +349,13 @@ gg_status gg_masked_forward(const void* A, const void* W, const int32_t* masked_
   if (mmax == 0) return GG_OK;
   if (A == nullptr || out == nullptr) return GG_ERR_INVALID_ARG;
   if (!aligned16(A) || !aligned16(W) || !aligned16(out)) return GG_ERR_UNSUPPORTED;
+  const bool chunked = (N % 64) == 0;
   CUtensorMap ma, mb;
-  if (!map_2d(&ma, A, (int64_t)E * mmax, K, 64, gg::BM) || !map_w(&mb, W, E, K, N, 64, 64))
+  if (!map_2d(&ma, A, (int64_t)E * mmax, K, 64, gg::BM)) return GG_ERR_CUDA;
+  if (chunked ? !map_w_chunked(&mb, W, E, K, N, 64, kBN / 64) : !map_w(&mb, W, E, K, N, 64, 64))
     return GG_ERR_CUDA;
   gg::Params p = base_params(masked_m, out, dev_status, (int64_t)E * mmax, E);
+  p.b_chunked = chunked ? 1 : 0;
   p.mmax = (int32_t)mmax;
   p.red_len = (int32_t)K;
   p.out_cols = (int32_t)N;

@@ -45,6 +45,35 @@ constexpr int BK = 64;          // reduction elements per stage (128 bytes of bf
 constexpr int UMMA_K = 16;      // reduction per tcgen05.mma for 16-bit inputs
 constexpr int NUM_THREADS = 192;
 
+// L2 eviction priority of the TMA loads: 0 normal, 1 evict-first, 2 evict-last.
+//   GG_L2_TOKENS   token-major operand of forward/dgrad/masked (A or dY), reused by the
+//                  N-tiles of one row band that run at the same time
+//   GG_L2_WEIGHTS  W[e], reused by every row band of group e
+//   GG_L2_WGRAD    both operands of wgrad
+#ifndef GG_L2_TOKENS
+#define GG_L2_TOKENS 1
+#endif
+#ifndef GG_L2_WEIGHTS
+#define GG_L2_WEIGHTS 2
+#endif
+#ifndef GG_L2_WGRAD
+#define GG_L2_WGRAD 2
+#endif
+// tcgen05 fence after every stage's full-barrier wait (the operands were written by TMA and
+// are ordered by the barrier itself; 0 leaves the fence out).
+#ifndef GG_FENCE_PER_STAGE
+#define GG_FENCE_PER_STAGE 1
+#endif
+// Longest suspension of one mbarrier probe (ns); the thread wakes early when the phase
+// completes. It also bounds how late an aborting role notices the abort flag.
+#ifndef GG_WAIT_SLICE_NS
+#define GG_WAIT_SLICE_NS 200000
+#endif
+// Back-off (ns) of the epilogue warps while they wait for an accumulator (0 = spin).
+#ifndef GG_EPI_BACKOFF_NS
+#define GG_EPI_BACKOFF_NS 0
+#endif
+
 // Device status bits (same values as the public header).
 constexpr int DEV_BAD_OFFSETS = 0x1;
 constexpr int DEV_BAD_MASKED_M = 0x2;
@@ -63,6 +92,10 @@ struct Params {
   int32_t wg_K;            // Wgrad: K (rows of each dW[e])
   uint64_t watchdog_ns;
   int32_t debug_flags;     // bit 0: CTA 0 skips its first load (watchdog test)
+  // 1 when the map of that operand covers all 64-wide chunks of a stage in one box (a
+  // dimension split as [.., dim/64, 64]); 0 when each chunk is its own box.
+  int32_t a_chunked;
+  int32_t b_chunked;
 };
 
 template <int BN, int STAGES, bool PAIR>
@@ -74,7 +107,8 @@ struct Layout {
   static constexpr uint32_t OFF_A = 0;
   static constexpr uint32_t OFF_B = STAGES * A_BYTES;
   static constexpr uint32_t OFF_BAR = STAGES * STAGE_BYTES;
-  static constexpr uint32_t NUM_BARS = 2 * STAGES + 5;  // full, empty, tfull x2, tempty x2, fin
+  // full, empty, landed (wgrad tail blocks) per stage; tfull x2, tempty x2, fin
+  static constexpr uint32_t NUM_BARS = 3 * STAGES + 5;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr uint32_t OFF_TAB = OFF_MISC + 16;
   static constexpr uint32_t TMEM_COLS = 2 * BN;
@@ -99,6 +133,7 @@ struct Tile {
 struct Shared {
   uint64_t* full;
   uint64_t* empty;
+  uint64_t* landed;
   uint64_t* tfull;
   uint64_t* tempty;
   uint64_t* fin;
@@ -115,35 +150,45 @@ __device__ __forceinline__ void set_status(const Params& p, int bits) {
   if (p.status != nullptr) atomicOr(p.status, bits);
 }
 
-// Bounded wait on one phase of an mbarrier. Returns false when the CTA is aborting or the
-// watchdog expired (then the abort flag and GG_DEV_TIMEOUT are set). `cluster` selects
-// acquire at cluster scope, for barriers that receive arrivals from the peer CTA.
-__device__ __noinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, const Shared& sh,
-                                          const Params& p, bool honour_abort,
-                                          bool cluster = false) {
-  auto probe = [&]() {
-    return cluster ? ptx::mbar_try_wait_cluster(bar, parity) : ptx::mbar_try_wait(bar, parity);
-  };
-  if (probe()) return true;
+// Bounded wait on one phase of an mbarrier, slow path: probes until the phase completes,
+// the CTA aborts, or the watchdog expires (then the abort flag and GG_DEV_TIMEOUT are set).
+// Each probe suspends the thread until the phase completes or about GG_WAIT_SLICE_NS pass.
+// `cluster` selects acquire at cluster scope, for barriers that receive arrivals from the
+// peer CTA.
+__device__ __noinline__ bool wait_slow(uint64_t* bar, uint32_t parity, const Shared& sh,
+                                       const Params& p, bool honour_abort, bool cluster,
+                                       uint32_t backoff_ns) {
   const uint64_t t0 = ptx::globaltimer();
-  for (uint32_t i = 1;; ++i) {
-    if (probe()) return true;
-    if ((i & 31u) == 0u) {
-      if (honour_abort && *sh.abort_flag) return false;
-      if (ptx::globaltimer() - t0 > p.watchdog_ns) {
-        *sh.abort_flag = 1;
-        set_status(p, DEV_TIMEOUT);
-        return false;
-      }
+  for (;;) {
+    if (backoff_ns) __nanosleep(backoff_ns);
+    const bool done = cluster ? ptx::mbar_try_wait_cluster(bar, parity, GG_WAIT_SLICE_NS)
+                              : ptx::mbar_try_wait(bar, parity, GG_WAIT_SLICE_NS);
+    if (done) return true;
+    if (honour_abort && *sh.abort_flag) return false;
+    if (ptx::globaltimer() - t0 > p.watchdog_ns) {
+      *sh.abort_flag = 1;
+      set_status(p, DEV_TIMEOUT);
+      return false;
     }
   }
 }
 
+// Bounded wait: one inline probe (the common case on a busy pipeline), then the slow path.
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, const Shared& sh,
+                                             const Params& p, bool honour_abort,
+                                             bool cluster = false, uint32_t backoff_ns = 0) {
+  const bool done = cluster ? ptx::mbar_try_wait_cluster(bar, parity, GG_WAIT_SLICE_NS)
+                            : ptx::mbar_try_wait(bar, parity, GG_WAIT_SLICE_NS);
+  if (done) return true;
+  return wait_slow(bar, parity, sh, p, honour_abort, cluster, backoff_ns);
+}
+
 // Single-lane wait whose outcome every lane of the warp shares.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const Shared& sh,
-                                          const Params& p, bool cluster) {
+                                          const Params& p, bool cluster,
+                                          uint32_t backoff_ns = 0) {
   bool ok = true;
-  if (ptx::lane_id() == 0) ok = wait_bounded(bar, parity, sh, p, true, cluster);
+  if (ptx::lane_id() == 0) ok = wait_bounded(bar, parity, sh, p, true, cluster, backoff_ns);
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
@@ -307,9 +352,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   sh.full = bars;
   sh.empty = bars + STAGES;
-  sh.tfull = bars + 2 * STAGES;
-  sh.tempty = bars + 2 * STAGES + 2;
-  sh.fin = bars + 2 * STAGES + 4;
+  sh.landed = bars + 2 * STAGES;
+  sh.tfull = bars + 3 * STAGES;
+  sh.tempty = bars + 3 * STAGES + 2;
+  sh.fin = bars + 3 * STAGES + 4;
   sh.tmem_base = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   sh.abort_flag = reinterpret_cast<volatile int32_t*>(smem + L::OFF_MISC + 4);
   sh.total = reinterpret_cast<int32_t*>(smem + L::OFF_MISC + 8);
@@ -330,6 +376,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int s = 0; s < STAGES; ++s) {
       ptx::mbar_init(&sh.full[s], 1);
       ptx::mbar_init(&sh.empty[s], 1);
+      ptx::mbar_init(&sh.landed[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       ptx::mbar_init(&sh.tfull[a], 1);
@@ -364,170 +411,200 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      const uint64_t pol_stream = ptx::policy_evict_first();
-      const uint64_t pol_keep = ptx::policy_evict_last();
-      uint32_t stage = 0, phase = 0;
-      uint32_t armed = 0, armed_par = 0;  // per-stage: loads in flight, and their phase
-      bool skip_first = (p.debug_flags & 1) && blockIdx.x == 0;
-      bool ok = true;
-      const int32_t row_off = (int32_t)rank * BM;       // this CTA's rows of a pair tile
-      const int32_t col_off = (int32_t)rank * L::B_COLS;  // this CTA's columns of B
-      for (int32_t t = unit0; t < total && ok; t += units) {
-        const Tile tl = decode_tile<MODE, BN, TM>(t, p, sh);
-        for (int32_t kb = 0; kb < tl.kblocks; ++kb) {
-          if (!wait_bounded(&sh.empty[stage], phase ^ 1u, sh, p, true)) { ok = false; break; }
+    // The whole warp walks the tile list; lane 0 waits and issues the loads. In wgrad the
+    // warp also zeroes the rows of a group's last, partial stage that lie past the group.
+    const uint64_t pol_tok = ptx::l2_policy<GG_L2_TOKENS>();
+    const uint64_t pol_w = ptx::l2_policy<GG_L2_WEIGHTS>();
+    const uint64_t pol_wg = ptx::l2_policy<GG_L2_WGRAD>();
+    uint32_t stage = 0, phase = 0;
+    uint32_t armed = 0, armed_par = 0;  // per stage: loads in flight on full[], their phase
+    uint32_t landed_par = 0;            // per stage: next phase of landed[]
+    bool skip_first = (p.debug_flags & 1) && blockIdx.x == 0;
+    bool ok = true;
+    const int32_t row_off = (int32_t)rank * BM;         // this CTA's rows of a pair tile
+    const int32_t col_off = (int32_t)rank * L::B_COLS;  // this CTA's columns of B
+    for (int32_t t = unit0; t < total && ok; t += units) {
+      const Tile tl = decode_tile<MODE, BN, TM>(t, p, sh);
+      for (int32_t kb = 0; kb < tl.kblocks; ++kb) {
+        if (!warp_wait(&sh.empty[stage], phase ^ 1u, sh, p, false)) { ok = false; break; }
+        uint8_t* sA = smem + L::OFF_A + stage * L::A_BYTES;
+        uint8_t* sB = smem + L::OFF_B + stage * L::B_BYTES;
+        uint64_t* fb = &sh.full[stage];
+        int32_t rem = BK;  // wgrad: rows of the group in this stage
+        if constexpr (MODE == Mode::Wgrad) rem = tl.tok_len - kb * BK;
+        const bool tail = MODE == Mode::Wgrad && rem < BK;
+        if (lane == 0) {
           armed &= ~(1u << stage);
-          uint8_t* sA = smem + L::OFF_A + stage * L::A_BYTES;
-          uint8_t* sB = smem + L::OFF_B + stage * L::B_BYTES;
-          uint64_t* fb = &sh.full[stage];
           if (skip_first) {
-            skip_first = false;  // watchdog test: never arm this stage
+            skip_first = false;  // watchdog test: this stage is never armed
           } else if constexpr (PAIR) {
             // the leader's full barrier counts the bytes of both CTAs
             const uint32_t fb_leader = ptx::mapa(ptx::smem_u32(fb), 0);
             if (leader) ptx::mbar_arrive_expect_tx(fb, 2 * L::STAGE_BYTES);
-            ptx::tma_load_2d_pair(sA, &mapA, fb_leader, kb * BK, tl.a_row0 + row_off,
-                                  pol_stream);
+            ptx::tma_load_2d_pair(sA, &mapA, fb_leader, kb * BK, tl.a_row0 + row_off, pol_tok);
             if constexpr (MODE == Mode::Dgrad) {
-              ptx::tma_load_3d_pair(sB, &mapB, fb_leader, kb * BK, tl.n0 + col_off, tl.e,
-                                    pol_keep);
+              ptx::tma_load_3d_pair(sB, &mapB, fb_leader, kb * BK, tl.n0 + col_off, tl.e, pol_w);
+            } else if (p.b_chunked) {
+              ptx::tma_load_4d_pair(sB, &mapB, fb_leader, 0, kb * BK, (tl.n0 + col_off) / 64,
+                                    tl.e, pol_w);
             } else {
 #pragma unroll
               for (int j = 0; j < L::B_COLS / 64; ++j)
                 ptx::tma_load_3d_pair(sB + j * 8192, &mapB, fb_leader, tl.n0 + col_off + j * 64,
-                                      kb * BK, tl.e, pol_keep);
+                                      kb * BK, tl.e, pol_w);
             }
             if (leader) {
               armed |= 1u << stage;
               armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
             }
           } else {
-            ptx::mbar_arrive_expect_tx(fb, L::STAGE_BYTES);
+            // a wgrad tail stage lands on landed[] first; full[] completes after the fix-up
+            uint64_t* lb = tail ? &sh.landed[stage] : fb;
+            ptx::mbar_arrive_expect_tx(lb, L::STAGE_BYTES);
             if constexpr (MODE == Mode::Forward || MODE == Mode::Masked) {
-              ptx::tma_load_2d(sA, &mapA, fb, kb * BK, tl.a_row0, pol_stream);
+              ptx::tma_load_2d(sA, &mapA, lb, kb * BK, tl.a_row0, pol_tok);
+              if (p.b_chunked) {
+                ptx::tma_load_4d(sB, &mapB, lb, 0, kb * BK, tl.n0 / 64, tl.e, pol_w);
+              } else {
 #pragma unroll
-              for (int j = 0; j < BN / 64; ++j)
-                ptx::tma_load_3d(sB + j * 8192, &mapB, fb, tl.n0 + j * 64, kb * BK, tl.e,
-                                 pol_keep);
+                for (int j = 0; j < BN / 64; ++j)
+                  ptx::tma_load_3d(sB + j * 8192, &mapB, lb, tl.n0 + j * 64, kb * BK, tl.e, pol_w);
+              }
             } else if constexpr (MODE == Mode::Dgrad) {
-              ptx::tma_load_2d(sA, &mapA, fb, kb * BK, tl.a_row0, pol_stream);
-              ptx::tma_load_3d(sB, &mapB, fb, kb * BK, tl.n0, tl.e, pol_keep);
+              ptx::tma_load_2d(sA, &mapA, lb, kb * BK, tl.a_row0, pol_tok);
+              ptx::tma_load_3d(sB, &mapB, lb, kb * BK, tl.n0, tl.e, pol_w);
             } else {  // Wgrad
               const int32_t r = tl.tok0 + kb * BK;
+              if (p.a_chunked) {
+                ptx::tma_load_3d(sA, &mapA, lb, 0, r, tl.k0 / 64, pol_wg);
+              } else {
 #pragma unroll
-              for (int j = 0; j < 2; ++j)
-                ptx::tma_load_2d(sA + j * 8192, &mapA, fb, tl.k0 + j * 64, r, pol_keep);
+                for (int j = 0; j < 2; ++j)
+                  ptx::tma_load_2d(sA + j * 8192, &mapA, lb, tl.k0 + j * 64, r, pol_wg);
+              }
+              if (p.b_chunked) {
+                ptx::tma_load_3d(sB, &mapB, lb, 0, r, tl.n0 / 64, pol_wg);
+              } else {
 #pragma unroll
-              for (int j = 0; j < BN / 64; ++j)
-                ptx::tma_load_2d(sB + j * 8192, &mapB, fb, tl.n0 + j * 64, r, pol_keep);
+                for (int j = 0; j < BN / 64; ++j)
+                  ptx::tma_load_2d(sB + j * 8192, &mapB, lb, tl.n0 + j * 64, r, pol_wg);
+              }
             }
-            armed |= 1u << stage;
-            armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+            if (!tail) {
+              armed |= 1u << stage;
+              armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+            }
           }
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
+        if constexpr (MODE == Mode::Wgrad) {
+          if (tail) {
+            // Rows [rem, ceil16(rem)) of this stage belong to the next group (or to no group):
+            // zero them in both operands so they add nothing; the MMA reads no row past
+            // ceil16(rem). A token row is one 128-byte line of every 64-wide chunk.
+            const uint32_t lp = (landed_par >> stage) & 1u;
+            landed_par ^= 1u << stage;
+            if (!warp_wait(&sh.landed[stage], lp, sh, p, false)) { ok = false; break; }
+            const int nsub = (rem + UMMA_K - 1) / UMMA_K;
+            const int zrows = nsub * UMMA_K - rem;
+            const int lines_a = zrows * 2, lines_b = zrows * (BN / 64);
+            for (int i = (int)lane; i < (lines_a + lines_b) * 8; i += 32) {
+              const int line = i >> 3, part = i & 7;
+              uint8_t* dst;
+              if (line < lines_a) {
+                dst = sA + (line / zrows) * 8192 + (rem + line % zrows) * 128 + part * 16;
+              } else {
+                const int l2 = line - lines_a;
+                dst = sB + (l2 / zrows) * 8192 + (rem + l2 % zrows) * 128 + part * 16;
+              }
+              *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+            }
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(fb);
+          }
+        }
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
-      // Let every load this thread armed land before the CTA can exit (on the normal path
-      // these phases have completed already; after an abort some may still be in flight).
-      // A pair follower's loads complete on the leader's barriers; they were issued at least
-      // one watchdog period before any abort could end this CTA.
+    }
+    // Let every load this warp armed land before the CTA can exit (on the normal path these
+    // phases have completed already; after an abort some may still be in flight). A pair
+    // follower's loads complete on the leader's barriers; they were issued at least one
+    // watchdog period before any abort could end this CTA.
+    if (lane == 0)
       for (int s = 0; s < STAGES; ++s)
         if (armed & (1u << s)) wait_bounded(&sh.full[s], (armed_par >> s) & 1u, sh, p, false);
-    }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (pair leader)
-    if (leader) {
+    // ------------------------------------------------------------ MMA issuer
+    // One lane of the pair leader issues every MMA; the loop carries no warp-wide
+    // synchronisation so that issue keeps ahead of the tensor pipe.
+    if (leader && lane == 0) {
+      // descriptor deltas per 16-element reduction step (address field is in 16-byte units)
+      constexpr uint64_t A_STEP = A_MN ? (2048u >> 4) : (32u >> 4);
+      constexpr uint64_t B_STEP = B_MN ? (2048u >> 4) : (32u >> 4);
+      const uint32_t a_lbo = A_MN ? 8192u : 16u, b_lbo = B_MN ? 8192u : 16u;
       uint32_t stage = 0, phase = 0, acc_iter = 0;
       bool ok = true;
       for (int32_t t = unit0; t < total && ok; t += units) {
         const Tile tl = decode_tile<MODE, BN, TM>(t, p, sh);
         if (tl.kblocks == 0) continue;  // Wgrad of an empty expert: the epilogue writes zeros
         const uint32_t a = acc_iter & 1u;
-        if (!warp_wait(&sh.tempty[a], ((acc_iter >> 1) & 1u) ^ 1u, sh, p, PAIR)) {
+        if (!wait_bounded(&sh.tempty[a], ((acc_iter >> 1) & 1u) ^ 1u, sh, p, true, PAIR)) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + a * BN;
         for (int32_t kb = 0; kb < tl.kblocks; ++kb) {
-          if (!warp_wait(&sh.full[stage], phase, sh, p, false)) { ok = false; break; }
+          if (!wait_bounded(&sh.full[stage], phase, sh, p, true)) { ok = false; break; }
+#if GG_FENCE_PER_STAGE
           ptx::tc_fence_after();
-          uint8_t* sA = smem + L::OFF_A + stage * L::A_BYTES;
-          uint8_t* sB = smem + L::OFF_B + stage * L::B_BYTES;
+#endif
           int nsub = BK / UMMA_K;
           if constexpr (MODE == Mode::Wgrad) {
-            const int32_t rem = tl.tok_len - kb * BK;  // rows of this group in the stage
-            if (rem < BK) {
-              nsub = (rem + UMMA_K - 1) / UMMA_K;
-              // Rows [rem, nsub*16) belong to the next group (or to no group): zero them in
-              // both operands so they add nothing. Each token row is one 128-byte line of
-              // every 64-wide chunk.
-              const int zrows = nsub * UMMA_K - rem;
-              const int lines_a = zrows * 2, lines_b = zrows * (BN / 64);
-              for (int i = (int)lane; i < (lines_a + lines_b) * 8; i += 32) {
-                const int line = i >> 3, part = i & 7;
-                uint8_t* dst;
-                if (line < lines_a) {
-                  const int c = line / zrows, rr = rem + line % zrows;
-                  dst = sA + c * 8192 + rr * 128 + part * 16;
-                } else {
-                  const int l2 = line - lines_a;
-                  const int c = l2 / zrows, rr = rem + l2 % zrows;
-                  dst = sB + c * 8192 + rr * 128 + part * 16;
-                }
-                *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
-              }
-              ptx::fence_proxy_async_smem();
-              __syncwarp();
-            }
+            const int32_t rem = tl.tok_len - kb * BK;
+            if (rem < BK) nsub = (rem + UMMA_K - 1) / UMMA_K;
           }
-          if (lane == 0) {
-            const uint32_t a_base = ptx::smem_u32(sA), b_base = ptx::smem_u32(sB);
-            for (int k = 0; k < nsub; ++k) {
-              uint64_t adesc, bdesc;
-              if constexpr (A_MN) adesc = ptx::smem_desc_sw128(a_base + k * 2048, 8192, 1024);
-              else                adesc = ptx::smem_desc_sw128(a_base + k * 32, 16, 1024);
-              if constexpr (B_MN) bdesc = ptx::smem_desc_sw128(b_base + k * 2048, 8192, 1024);
-              else                bdesc = ptx::smem_desc_sw128(b_base + k * 32, 16, 1024);
+          const uint64_t adesc = ptx::smem_desc_sw128(
+              ptx::smem_u32(smem + L::OFF_A + stage * L::A_BYTES), a_lbo, 1024);
+          const uint64_t bdesc = ptx::smem_desc_sw128(
+              ptx::smem_u32(smem + L::OFF_B + stage * L::B_BYTES), b_lbo, 1024);
+#pragma unroll
+          for (int k = 0; k < BK / UMMA_K; ++k) {
+            if (k < nsub) {
               const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
-              if constexpr (PAIR) ptx::mma_bf16_pair(d_tmem, adesc, bdesc, IDESC, acc);
-              else                ptx::mma_bf16(d_tmem, adesc, bdesc, IDESC, acc);
-            }
-            // free the stage (in both CTAs of a pair) once these MMAs are done
-            if constexpr (PAIR) {
-              const uint32_t eb = ptx::smem_u32(&sh.empty[stage]);
-              ptx::mma_commit_pair(ptx::mapa(eb, 0));
-              ptx::mma_commit_pair(ptx::mapa(eb, 1));
-            } else {
-              ptx::mma_commit(&sh.empty[stage]);
+              if constexpr (PAIR)
+                ptx::mma_bf16_pair(d_tmem, adesc + k * A_STEP, bdesc + k * B_STEP, IDESC, acc);
+              else
+                ptx::mma_bf16(d_tmem, adesc + k * A_STEP, bdesc + k * B_STEP, IDESC, acc);
             }
           }
-          __syncwarp();
+          // free the stage (in both CTAs of a pair) once these MMAs are done
+          if constexpr (PAIR) {
+            const uint32_t eb = ptx::smem_u32(&sh.empty[stage]);
+            ptx::mma_commit_pair(ptx::mapa(eb, 0));
+            ptx::mma_commit_pair(ptx::mapa(eb, 1));
+          } else {
+            ptx::mma_commit(&sh.empty[stage]);
+          }
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        if (lane == 0) {
-          if constexpr (PAIR) {
-            const uint32_t fb = ptx::smem_u32(&sh.tfull[a]);
-            ptx::mma_commit_pair(ptx::mapa(fb, 0));
-            ptx::mma_commit_pair(ptx::mapa(fb, 1));
-          } else {
-            ptx::mma_commit(&sh.tfull[a]);
-          }
+        if constexpr (PAIR) {
+          const uint32_t fb = ptx::smem_u32(&sh.tfull[a]);
+          ptx::mma_commit_pair(ptx::mapa(fb, 0));
+          ptx::mma_commit_pair(ptx::mapa(fb, 1));
+        } else {
+          ptx::mma_commit(&sh.tfull[a]);
         }
-        __syncwarp();
         ++acc_iter;
       }
       // every MMA issued by this CTA completes before tensor memory is released
-      if (lane == 0) {
-        if constexpr (PAIR) ptx::mma_commit_pair(ptx::mapa(ptx::smem_u32(sh.fin), 0));
-        else                ptx::mma_commit(sh.fin);
-        wait_bounded(sh.fin, 0, sh, p, false);
-      }
-      __syncwarp();
+      if constexpr (PAIR) ptx::mma_commit_pair(ptx::mapa(ptx::smem_u32(sh.fin), 0));
+      else                ptx::mma_commit(sh.fin);
+      wait_bounded(sh.fin, 0, sh, p, false);
     }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
     const uint32_t q = warp & 3u;  // TMEM lane quadrant this warp may access
@@ -555,7 +632,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         continue;
       }
       const uint32_t a = acc_iter & 1u;
-      if (!warp_wait(&sh.tfull[a], (acc_iter >> 1) & 1u, sh, p, false)) break;
+      if (!warp_wait(&sh.tfull[a], (acc_iter >> 1) & 1u, sh, p, false, GG_EPI_BACKOFF_NS)) break;
       ptx::tc_fence_after();
       const uint32_t taddr = tmem_base + ((q * 32u) << 16) + a * BN;
 #pragma unroll 1

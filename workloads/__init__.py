@@ -41,6 +41,9 @@ CONFIGS = {
     "downproj": dict(E=32, K=2048, N=7168, T=65536, seed=4),
     "large": dict(E=16, K=6144, N=4096, T=262144, seed=5),
     "large_unaligned": dict(E=16, K=6144, N=4096, T=262144, seed=5),
+    # two experts of the large shape (1.2 GB on the device): the profiling case of the
+    # large-shape kernels
+    "large_e2": dict(E=2, K=6144, N=4096, T=32768, seed=6),
 }
 
 
@@ -83,7 +86,7 @@ def group_sizes(name: str, seed: Optional[int] = None) -> np.ndarray:
                 sizes = np.zeros(E, dtype=np.int64)
                 sizes[live] = s
                 return sizes
-    if name == "large":
+    if name in ("large", "large_e2"):
         return np.full(E, T // E, dtype=np.int64)
     if name == "large_unaligned":
         d = rng.integers(1, 128, E // 2)
