@@ -36,8 +36,16 @@ UNIT = "TFLOP/s"
 
 # DRAM bytes per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum), keyed by
 # kernel and workload, valid only for the kernel sources whose hash is recorded with them.
-NCU_TRAFFIC = {}
-NCU_TRAFFIC_SRC_HASH = None
+# Captured with: ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum
+#   --clock-control none -k regex:grouped_gemm -s 12 -c 4 python bench.py --steps 1 --warmup 3
+#   --no-e2e --no-cpu   (see profiles/grouped_gemm_large_launch_list.md)
+NCU_TRAFFIC = {
+    ("forward", "large"): 34.505e9,
+    ("dgrad", "large"): 30.346e9,
+    ("wgrad", "large"): 17.358e9,
+    ("masked", "large"): 0.0234e9,
+}
+NCU_TRAFFIC_SRC_HASH = "caa0295f233c78fb"
 
 
 def kernel_source_hash() -> str:
