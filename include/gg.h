@@ -137,7 +137,7 @@ GG_API uint64_t gg_set_watchdog_ns(uint64_t ns);
    GG_DEV_TIMEOUT. No GPU fault is involved. Returns the previous setting. */
 GG_API int gg_testing_skip_first_load(int enable);
 
-/* Test hook: choose the launch shape of gg_forward and gg_dgrad for later calls:
+/* Test hook: choose the launch shape of gg_forward, gg_dgrad and gg_wgrad for later calls:
    0 = automatic (CTA pairs when rows_alloc >= 512*E), 1 = single CTAs (128-row tiles),
    2 = CTA pairs (256-row tiles on two SMs). Results are the same up to rounding order.
    Returns the previous setting. */

@@ -88,7 +88,7 @@ def testing_skip_first_load(enable: bool) -> bool:
 
 
 def testing_force_variant(variant: int) -> int:
-    """Test hook: 0 automatic, 1 single-CTA tiles, 2 CTA-pair tiles (forward and dgrad)."""
+    """Test hook: 0 automatic, 1 single-CTA tiles, 2 CTA-pair tiles (forward, dgrad, wgrad)."""
     return int(lib().gg_testing_force_variant(int(variant)))
 
 

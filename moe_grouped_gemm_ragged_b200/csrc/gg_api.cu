@@ -214,6 +214,11 @@ gg::Params base_params(const int32_t* groups, void* out, int32_t* status, int64_
   return p;
 }
 
+// 256-bit epilogue stores need every output row to start on a 32-byte boundary.
+void set_store_width(gg::Params* p, const void* out, int64_t cols) {
+  p->out_v8 = ((reinterpret_cast<uintptr_t>(out) & 31u) == 0 && cols % 16 == 0) ? 1 : 0;
+}
+
 gg_status check_common(int64_t rows_alloc, int64_t K, int64_t N, int32_t E,
                        const int32_t* groups, const int32_t* dev_status, DeviceInfo* di) {
   if (E < 1 || K < 1 || N < 1 || rows_alloc < 0 || groups == nullptr) return GG_ERR_INVALID_ARG;
@@ -270,6 +275,7 @@ gg_status gg_forward(const void* A, const void* W, const int32_t* offs, void* ou
   p.red_len = (int32_t)K;
   p.out_cols = (int32_t)N;
   p.b_chunked = chunked ? 1 : 0;
+  set_store_width(&p, out, N);
   if (pair) {
     const int64_t tiles = (cdiv(rows_alloc, 2 * gg::BM) + E) * cdiv(N, kBN);
     return launch<Mode::Forward, kBN, kPairStages, true>(ma, mb, p, tiles, di, stream);
@@ -296,6 +302,7 @@ gg_status gg_dgrad(const void* dY, const void* W, const int32_t* offs, void* dX,
   gg::Params p = base_params(offs, dX, dev_status, rows_alloc, E);
   p.red_len = (int32_t)N;
   p.out_cols = (int32_t)K;
+  set_store_width(&p, dX, K);
   if (pair) {
     const int64_t tiles = (cdiv(rows_alloc, 2 * gg::BM) + E) * cdiv(K, kBN);
     return launch<Mode::Dgrad, kBN, kPairStages, true>(ma, mb, p, tiles, di, stream);
@@ -321,18 +328,27 @@ gg_status gg_wgrad(const void* A, const void* dY, const int32_t* offs, void* dW,
     dY = dW;
   }
   const bool a_chunked = (K % 64) == 0, b_chunked = (N % 64) == 0;
+  // wgrad stays on single CTAs unless forced: measured faster on long groups (large shape
+  // 1159 vs 909 TFLOP/s) and equal on short ones
+  const bool pair = g_force_variant.load() == 2;
+  const uint32_t bcols = pair ? kBN / 2 : kBN;  // dY columns one CTA loads per stage
   CUtensorMap ma, mb;
   if (a_chunked ? !map_2d_chunked(&ma, A, rows_alloc, K, 64, gg::BM / 64)
                 : !map_2d(&ma, A, rows_alloc, K, 64, 64))
     return GG_ERR_CUDA;
-  if (b_chunked ? !map_2d_chunked(&mb, dY, rows_alloc, N, 64, kBN / 64)
+  if (b_chunked ? !map_2d_chunked(&mb, dY, rows_alloc, N, 64, bcols / 64)
                 : !map_2d(&mb, dY, rows_alloc, N, 64, 64))
     return GG_ERR_CUDA;
   gg::Params p = base_params(offs, dW, dev_status, rows_alloc, E);
   p.out_cols = (int32_t)N;
   p.wg_K = (int32_t)K;
+  set_store_width(&p, dW, N);
   p.a_chunked = a_chunked ? 1 : 0;
   p.b_chunked = b_chunked ? 1 : 0;
+  if (pair) {
+    const int64_t tiles = (int64_t)E * cdiv(K, 2 * gg::BM) * cdiv(N, kBN);
+    return launch<Mode::Wgrad, kBN, kPairStages, true>(ma, mb, p, tiles, di, stream);
+  }
   const int64_t tiles = (int64_t)E * cdiv(K, gg::BM) * cdiv(N, kBN);
   return launch<Mode::Wgrad, kBN, kStages, false>(ma, mb, p, tiles, di, stream);
 }
@@ -359,6 +375,7 @@ gg_status gg_masked_forward(const void* A, const void* W, const int32_t* masked_
   p.mmax = (int32_t)mmax;
   p.red_len = (int32_t)K;
   p.out_cols = (int32_t)N;
+  set_store_width(&p, out, N);
   const int64_t tiles = (int64_t)E * cdiv(mmax, gg::BM) * cdiv(N, kBN);
   return launch<Mode::Masked, kBN, kStages, false>(ma, mb, p, tiles, di, stream);
 }

@@ -18,8 +18,10 @@
 //   warp 0      TMA producer: one lane arms a stage barrier and issues the tensor loads
 //   warp 1      tensor-memory owner and MMA issuer: one lane issues tcgen05.mma into a
 //               double-buffered fp32 accumulator in TMEM (2 x BN columns)
-//   warps 2..5  epilogue: tcgen05.ld of their 32-lane quadrant, fp32 -> bf16 (nearest even),
-//               predicated 16-byte stores of the rows inside the group and columns < N
+//   warps 2..9  epilogue: two warps per 32-lane TMEM quadrant, each owning half of the
+//               columns; tcgen05.ld (double-buffered registers), fp32 -> bf16 (nearest
+//               even), predicated 32- or 16-byte stores of rows inside the group, columns < N
+//   warp 10     wgrad only: zeroes the rows of a group's last stage that lie past the group
 //
 // Shared-memory stages use the 128-byte swizzle that both TMA and tcgen05 understand:
 //   K-major operand  (reduction contiguous):  [rows][64 elements = 128 B]
@@ -43,7 +45,9 @@ enum class Mode : int { Forward = 0, Dgrad = 1, Wgrad = 2, Masked = 3 };
 constexpr int BM = 128;         // tile rows (TMEM lanes)
 constexpr int BK = 64;          // reduction elements per stage (128 bytes of bf16)
 constexpr int UMMA_K = 16;      // reduction per tcgen05.mma for 16-bit inputs
-constexpr int NUM_THREADS = 192;
+constexpr int EPI_WARPS = 8;      // two per TMEM lane quadrant, each owning half the columns
+constexpr int FIX_WARP = 2 + EPI_WARPS;  // wgrad: zeroes the rows of a group's last stage
+constexpr int NUM_THREADS = 32 * (FIX_WARP + 1);
 
 // L2 eviction priority of the TMA loads: 0 normal, 1 evict-first, 2 evict-last.
 //   GG_L2_TOKENS   token-major operand of forward/dgrad/masked (A or dY), reused by the
@@ -96,6 +100,7 @@ struct Params {
   // dimension split as [.., dim/64, 64]); 0 when each chunk is its own box.
   int32_t a_chunked;
   int32_t b_chunked;
+  int32_t out_v8;          // 1 when every output row starts 32-byte aligned (256-bit stores)
 };
 
 template <int BN, int STAGES, bool PAIR>
@@ -107,8 +112,8 @@ struct Layout {
   static constexpr uint32_t OFF_A = 0;
   static constexpr uint32_t OFF_B = STAGES * A_BYTES;
   static constexpr uint32_t OFF_BAR = STAGES * STAGE_BYTES;
-  // full, empty, landed (wgrad tail blocks) per stage; tfull x2, tempty x2, fin
-  static constexpr uint32_t NUM_BARS = 3 * STAGES + 5;
+  // full, empty, landed, fixed (wgrad tail blocks) per stage; tfull x2, tempty x2, fin
+  static constexpr uint32_t NUM_BARS = 4 * STAGES + 5;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr uint32_t OFF_TAB = OFF_MISC + 16;
   static constexpr uint32_t TMEM_COLS = 2 * BN;
@@ -134,6 +139,7 @@ struct Shared {
   uint64_t* full;
   uint64_t* empty;
   uint64_t* landed;
+  uint64_t* fixed;
   uint64_t* tfull;
   uint64_t* tempty;
   uint64_t* fin;
@@ -258,7 +264,7 @@ __device__ void build_table(const Params& p, const Shared& sh) {
   if (lane == 0) {
     if (bad) set_status(p, MODE == Mode::Masked ? DEV_BAD_MASKED_M : DEV_BAD_OFFSETS);
     if constexpr (MODE == Mode::Wgrad) {
-      const int32_t KT = (p.wg_K + BM - 1) / BM;
+      const int32_t KT = (p.wg_K + TM - 1) / TM;
       *sh.total = E * KT * NT;
     } else {
       *sh.total = tiles_carry;
@@ -286,7 +292,7 @@ __device__ __forceinline__ Tile decode_tile(int32_t t, const Params& p, const Sh
   Tile tl;
   const int32_t NT = (p.out_cols + BN - 1) / BN;
   if constexpr (MODE == Mode::Wgrad) {
-    const int32_t KT = (p.wg_K + BM - 1) / BM;
+    const int32_t KT = (p.wg_K + TM - 1) / TM;
     const int32_t per = KT * NT;
     const int32_t slot = t / per;
     const int32_t local = t - slot * per;
@@ -294,7 +300,7 @@ __device__ __forceinline__ Tile decode_tile(int32_t t, const Params& p, const Sh
     const int32_t nt = local - kt * NT;
     const int32_t e = sh.order[slot];
     tl.e = e;
-    tl.k0 = kt * BM;
+    tl.k0 = kt * TM;
     tl.n0 = nt * BN;
     tl.tok0 = sh.gstart[e];
     tl.tok_len = sh.gend[e] - sh.gstart[e];
@@ -334,7 +340,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   using L = Layout<BN, STAGES, PAIR>;
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN must be 64, 128, 192 or 256");
   static_assert(!PAIR || BN % 128 == 0, "a CTA pair splits BN into two multiples of 64");
-  static_assert(!(PAIR && MODE == Mode::Wgrad), "wgrad runs on single CTAs");
   static_assert(L::TMEM_COLS == 128 || L::TMEM_COLS == 256 || L::TMEM_COLS == 512,
                 "TMEM allocation must be a power of two");
   constexpr int TM = PAIR ? 2 * BM : BM;  // rows of a tile
@@ -342,7 +347,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   constexpr uint32_t A_MN = (MODE == Mode::Wgrad) ? 1u : 0u;
   constexpr uint32_t B_MN = (MODE == Mode::Dgrad) ? 0u : 1u;
   constexpr uint32_t IDESC = ptx::idesc_bf16_f32(TM, BN, A_MN, B_MN);
-  constexpr uint32_t EPI_ARRIVALS = PAIR ? 8u : 4u;  // one per epilogue warp of the tile
+  constexpr uint32_t EPI_ARRIVALS = (PAIR ? 2u : 1u) * EPI_WARPS;  // one per epilogue warp
+  // In a pair's wgrad, the follower signals its fixed-up half of a group's last stage on the
+  // leader's fixed[] barrier (a stage with whole rows only completes by its byte count).
+  constexpr bool PAIR_WGRAD = PAIR && MODE == Mode::Wgrad;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = ptx::smem_u32(smem_raw);
@@ -353,9 +361,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   sh.full = bars;
   sh.empty = bars + STAGES;
   sh.landed = bars + 2 * STAGES;
-  sh.tfull = bars + 3 * STAGES;
-  sh.tempty = bars + 3 * STAGES + 2;
-  sh.fin = bars + 3 * STAGES + 4;
+  sh.fixed = bars + 3 * STAGES;
+  sh.tfull = bars + 4 * STAGES;
+  sh.tempty = bars + 4 * STAGES + 2;
+  sh.fin = bars + 4 * STAGES + 4;
   sh.tmem_base = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   sh.abort_flag = reinterpret_cast<volatile int32_t*>(smem + L::OFF_MISC + 4);
   sh.total = reinterpret_cast<int32_t*>(smem + L::OFF_MISC + 8);
@@ -377,6 +386,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ptx::mbar_init(&sh.full[s], 1);
       ptx::mbar_init(&sh.empty[s], 1);
       ptx::mbar_init(&sh.landed[s], 1);
+      ptx::mbar_init(&sh.fixed[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       ptx::mbar_init(&sh.tfull[a], 1);
@@ -411,14 +421,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    // The whole warp walks the tile list; lane 0 waits and issues the loads. In wgrad the
-    // warp also zeroes the rows of a group's last, partial stage that lie past the group.
+    // The whole warp walks the tile list; lane 0 waits and issues the loads. A wgrad stage
+    // that ends its group lands on landed[] for the fix-up warp instead of on full[].
     const uint64_t pol_tok = ptx::l2_policy<GG_L2_TOKENS>();
     const uint64_t pol_w = ptx::l2_policy<GG_L2_WEIGHTS>();
     const uint64_t pol_wg = ptx::l2_policy<GG_L2_WGRAD>();
     uint32_t stage = 0, phase = 0;
     uint32_t armed = 0, armed_par = 0;  // per stage: loads in flight on full[], their phase
-    uint32_t landed_par = 0;            // per stage: next phase of landed[]
+    uint32_t armed_l = 0, armed_lpar = 0;  // the same for loads on landed[] (wgrad tails)
+    uint32_t landed_par = 0;  // per stage: phase of the next load on landed[]
+    auto lp_of = [&](uint32_t st) { return (landed_par >> st) & 1u; };
     bool skip_first = (p.debug_flags & 1) && blockIdx.x == 0;
     bool ok = true;
     const int32_t row_off = (int32_t)rank * BM;         // this CTA's rows of a pair tile
@@ -435,8 +447,51 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const bool tail = MODE == Mode::Wgrad && rem < BK;
         if (lane == 0) {
           armed &= ~(1u << stage);
+          armed_l &= ~(1u << stage);
           if (skip_first) {
             skip_first = false;  // watchdog test: this stage is never armed
+          } else if constexpr (PAIR && MODE == Mode::Wgrad) {
+            const int32_t r = tl.tok0 + kb * BK;
+            const int32_t ka = tl.k0 + row_off;  // this CTA's 128 columns of A (K)
+            const int32_t nb = tl.n0 + col_off;  // this CTA's columns of dY (N)
+            if (tail) {
+              // lands locally; the warp fixes it up and then arrives on the leader's barrier
+              uint64_t* lb = &sh.landed[stage];
+              ptx::mbar_arrive_expect_tx(lb, L::STAGE_BYTES);
+              armed_l |= 1u << stage;
+              armed_lpar = (armed_lpar & ~(1u << stage)) | (lp_of(stage) << stage);
+              if (p.a_chunked) {
+                ptx::tma_load_3d(sA, &mapA, lb, 0, r, ka / 64, pol_wg);
+              } else {
+                for (int j = 0; j < 2; ++j)
+                  ptx::tma_load_2d(sA + j * 8192, &mapA, lb, ka + j * 64, r, pol_wg);
+              }
+              if (p.b_chunked) {
+                ptx::tma_load_3d(sB, &mapB, lb, 0, r, nb / 64, pol_wg);
+              } else {
+                for (int j = 0; j < L::B_COLS / 64; ++j)
+                  ptx::tma_load_2d(sB + j * 8192, &mapB, lb, nb + j * 64, r, pol_wg);
+              }
+            } else {
+              const uint32_t fb_leader = ptx::mapa(ptx::smem_u32(fb), 0);
+              if (leader) ptx::mbar_arrive_expect_tx(fb, 2 * L::STAGE_BYTES);
+              if (p.a_chunked) {
+                ptx::tma_load_3d_pair(sA, &mapA, fb_leader, 0, r, ka / 64, pol_wg);
+              } else {
+                for (int j = 0; j < 2; ++j)
+                  ptx::tma_load_2d_pair(sA + j * 8192, &mapA, fb_leader, ka + j * 64, r, pol_wg);
+              }
+              if (p.b_chunked) {
+                ptx::tma_load_3d_pair(sB, &mapB, fb_leader, 0, r, nb / 64, pol_wg);
+              } else {
+                for (int j = 0; j < L::B_COLS / 64; ++j)
+                  ptx::tma_load_2d_pair(sB + j * 8192, &mapB, fb_leader, nb + j * 64, r, pol_wg);
+              }
+              if (leader) {
+                armed |= 1u << stage;
+                armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+              }
+            }
           } else if constexpr (PAIR) {
             // the leader's full barrier counts the bytes of both CTAs
             const uint32_t fb_leader = ptx::mapa(ptx::smem_u32(fb), 0);
@@ -493,36 +548,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (!tail) {
               armed |= 1u << stage;
               armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+            } else {
+              armed_l |= 1u << stage;
+              armed_lpar = (armed_lpar & ~(1u << stage)) | (lp_of(stage) << stage);
             }
           }
         }
-        if constexpr (MODE == Mode::Wgrad) {
-          if (tail) {
-            // Rows [rem, ceil16(rem)) of this stage belong to the next group (or to no group):
-            // zero them in both operands so they add nothing; the MMA reads no row past
-            // ceil16(rem). A token row is one 128-byte line of every 64-wide chunk.
-            const uint32_t lp = (landed_par >> stage) & 1u;
-            landed_par ^= 1u << stage;
-            if (!warp_wait(&sh.landed[stage], lp, sh, p, false)) { ok = false; break; }
-            const int nsub = (rem + UMMA_K - 1) / UMMA_K;
-            const int zrows = nsub * UMMA_K - rem;
-            const int lines_a = zrows * 2, lines_b = zrows * (BN / 64);
-            for (int i = (int)lane; i < (lines_a + lines_b) * 8; i += 32) {
-              const int line = i >> 3, part = i & 7;
-              uint8_t* dst;
-              if (line < lines_a) {
-                dst = sA + (line / zrows) * 8192 + (rem + line % zrows) * 128 + part * 16;
-              } else {
-                const int l2 = line - lines_a;
-                dst = sB + (l2 / zrows) * 8192 + (rem + l2 % zrows) * 128 + part * 16;
-              }
-              *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
-            }
-            ptx::fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(fb);
-          }
-        }
+        if (tail) landed_par ^= 1u << stage;
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
     }
@@ -531,8 +563,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // follower's loads complete on the leader's barriers; they were issued at least one
     // watchdog period before any abort could end this CTA.
     if (lane == 0)
-      for (int s = 0; s < STAGES; ++s)
+      for (int s = 0; s < STAGES; ++s) {
         if (armed & (1u << s)) wait_bounded(&sh.full[s], (armed_par >> s) & 1u, sh, p, false);
+        if (armed_l & (1u << s))
+          wait_bounded(&sh.landed[s], (armed_lpar >> s) & 1u, sh, p, false);
+      }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -544,6 +579,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       constexpr uint64_t B_STEP = B_MN ? (2048u >> 4) : (32u >> 4);
       const uint32_t a_lbo = A_MN ? 8192u : 16u, b_lbo = B_MN ? 8192u : 16u;
       uint32_t stage = 0, phase = 0, acc_iter = 0;
+      uint32_t fixed_par = 0;  // per stage: next phase of fixed[] (pair wgrad)
       bool ok = true;
       for (int32_t t = unit0; t < total && ok; t += units) {
         const Tile tl = decode_tile<MODE, BN, TM>(t, p, sh);
@@ -563,7 +599,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           int nsub = BK / UMMA_K;
           if constexpr (MODE == Mode::Wgrad) {
             const int32_t rem = tl.tok_len - kb * BK;
-            if (rem < BK) nsub = (rem + UMMA_K - 1) / UMMA_K;
+            if (rem < BK) {
+              nsub = (rem + UMMA_K - 1) / UMMA_K;
+              if constexpr (PAIR_WGRAD) {
+                // the follower's half of this stage is fixed up on its own schedule
+                const uint32_t fp = (fixed_par >> stage) & 1u;
+                fixed_par ^= 1u << stage;
+                if (!wait_bounded(&sh.fixed[stage], fp, sh, p, true, true)) { ok = false; break; }
+              }
+            }
           }
           const uint64_t adesc = ptx::smem_desc_sw128(
               ptx::smem_u32(smem + L::OFF_A + stage * L::A_BYTES), a_lbo, 1024);
@@ -605,9 +649,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       wait_bounded(sh.fin, 0, sh, p, false);
     }
     __syncwarp();
-  } else {
+  } else if (warp < FIX_WARP) {
     // ------------------------------------------------------------ epilogue
-    const uint32_t q = warp & 3u;  // TMEM lane quadrant this warp may access
+    const uint32_t q = warp & 3u;                 // TMEM lane quadrant this warp may access
+    constexpr int CW = BN / 2;                    // columns per epilogue warp
+    const int32_t c_off = ((int32_t)warp - 2) / 4 * CW;
     const int32_t row_in_tile = (int32_t)(rank * BM + q * 32 + lane);
     // tensor memory of this CTA's accumulator is released on the pair leader's barrier
     uint32_t tempty0 = ptx::smem_u32(&sh.tempty[0]), tempty1 = ptx::smem_u32(&sh.tempty[1]);
@@ -615,16 +661,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tempty0 = ptx::mapa(tempty0, 0);
       tempty1 = ptx::mapa(tempty1, 0);
     }
+    const bool v8 = p.out_v8 != 0;
     uint32_t acc_iter = 0;
     for (int32_t t = unit0; t < total; t += units) {
       const Tile tl = decode_tile<MODE, BN, TM>(t, p, sh);
       const int64_t orow = tl.row0 + row_in_tile;
       const bool row_ok = orow < tl.row_end;
       __nv_bfloat16* orow_ptr = p.out + orow * (int64_t)p.out_cols;
+      const int32_t col0 = tl.n0 + c_off;
       if (tl.kblocks == 0) {
         if (row_ok) {
-          for (int c = 0; c < BN; c += 8) {
-            const int32_t col = tl.n0 + c;
+          for (int c = 0; c < CW; c += 8) {
+            const int32_t col = col0 + c;
             if (col < p.out_cols)
               *reinterpret_cast<uint4*>(orow_ptr + col) = make_uint4(0u, 0u, 0u, 0u);
           }
@@ -634,26 +682,37 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t a = acc_iter & 1u;
       if (!warp_wait(&sh.tfull[a], (acc_iter >> 1) & 1u, sh, p, false, GG_EPI_BACKOFF_NS)) break;
       ptx::tc_fence_after();
-      const uint32_t taddr = tmem_base + ((q * 32u) << 16) + a * BN;
-#pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
-        uint32_t r[32];
-        ptx::tmem_ld_32x32b_x32(taddr + c, r);
+      const uint32_t taddr = tmem_base + ((q * 32u) << 16) + a * BN + (uint32_t)c_off;
+      // 32 columns per load; the next load is in flight while this chunk is stored
+      uint32_t r0[32], r1[32];
+      ptx::tmem_ld_32x32b_x32(taddr, r0);
+#pragma unroll
+      for (int c = 0; c < CW; c += 32) {
+        uint32_t(&cur)[32] = ((c / 32) & 1) ? r1 : r0;
+        uint32_t(&nxt)[32] = ((c / 32) & 1) ? r0 : r1;
         ptx::tmem_ld_wait();
+        if (c + 32 < CW) ptx::tmem_ld_32x32b_x32(taddr + c + 32, nxt);
         if (row_ok) {
+          uint32_t packed[16];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int32_t col = tl.n0 + c + j * 8;
-            if (col < p.out_cols) {
-              uint4 v;
-              uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+          for (int h = 0; h < 16; ++h) {
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(cur[2 * h]),
+                                                      __uint_as_float(cur[2 * h + 1]));
+            packed[h] = *reinterpret_cast<uint32_t*>(&b2);
+          }
+          if (v8) {
 #pragma unroll
-              for (int h = 0; h < 4; ++h) {
-                __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[j * 8 + 2 * h]),
-                                                          __uint_as_float(r[j * 8 + 2 * h + 1]));
-                w[h] = *reinterpret_cast<uint32_t*>(&b2);
-              }
-              *reinterpret_cast<uint4*>(orow_ptr + col) = v;
+            for (int j = 0; j < 2; ++j) {
+              const int32_t col = col0 + c + j * 16;
+              if (col < p.out_cols) ptx::st_global_v8(orow_ptr + col, packed + 8 * j);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int32_t col = col0 + c + j * 8;
+              if (col < p.out_cols)
+                *reinterpret_cast<uint4*>(orow_ptr + col) =
+                    make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
             }
           }
         }
@@ -665,6 +724,49 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         else                ptx::mbar_arrive(&sh.tempty[a]);
       }
       ++acc_iter;
+    }
+  } else if constexpr (MODE == Mode::Wgrad) {
+    // ------------------------------------------------------------ wgrad tail fix-up
+    // Walks the same stage sequence as the load warp. For a stage that ends its group, rows
+    // [rem, ceil16(rem)) belong to the next group (or to no group): they are zeroed in both
+    // operands so that they add nothing (the MMA reads no row past ceil16(rem)); a token row
+    // is one 128-byte line of every 64-wide chunk.
+    uint32_t stage = 0, landed_par = 0;
+    for (int32_t t = unit0; t < total; t += units) {
+      const Tile tl = decode_tile<MODE, BN, TM>(t, p, sh);
+      bool ok = true;
+      for (int32_t kb = 0; kb < tl.kblocks; ++kb) {
+        const int32_t rem = tl.tok_len - kb * BK;
+        if (rem < BK) {
+          const uint32_t lp = (landed_par >> stage) & 1u;
+          landed_par ^= 1u << stage;
+          if (!warp_wait(&sh.landed[stage], lp, sh, p, false)) { ok = false; break; }
+          uint8_t* sA = smem + L::OFF_A + stage * L::A_BYTES;
+          uint8_t* sB = smem + L::OFF_B + stage * L::B_BYTES;
+          const int nsub = (rem + UMMA_K - 1) / UMMA_K;
+          const int zrows = nsub * UMMA_K - rem;
+          const int lines_a = zrows * 2, lines_b = zrows * (L::B_COLS / 64);
+          for (int i = (int)lane; i < (lines_a + lines_b) * 8; i += 32) {
+            const int line = i >> 3, part = i & 7;
+            uint8_t* dst;
+            if (line < lines_a) {
+              dst = sA + (line / zrows) * 8192 + (rem + line % zrows) * 128 + part * 16;
+            } else {
+              const int l2 = line - lines_a;
+              dst = sB + (l2 / zrows) * 8192 + (rem + l2 % zrows) * 128 + part * 16;
+            }
+            *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+          }
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (leader) ptx::mbar_arrive(&sh.full[stage]);  // the leader's half completes full[]
+            else ptx::mbar_arrive_cluster(ptx::mapa(ptx::smem_u32(&sh.fixed[stage]), 0));
+          }
+        }
+        if (++stage == STAGES) stage = 0;
+      }
+      if (!ok) break;
     }
   }
 
