@@ -51,11 +51,12 @@ constexpr int NUM_THREADS = 32 * (FIX_WARP + 1);
 
 // L2 eviction priority of the TMA loads: 0 normal, 1 evict-first, 2 evict-last.
 //   GG_L2_TOKENS   token-major operand of forward/dgrad/masked (A or dY), reused by the
-//                  N-tiles of one row band that run at the same time
+//                  N-tiles of one row band that run at the same time (evict-first here
+//                  doubled the DRAM traffic of the large shape: 36 GB vs 18 GB per pass)
 //   GG_L2_WEIGHTS  W[e], reused by every row band of group e
 //   GG_L2_WGRAD    both operands of wgrad
 #ifndef GG_L2_TOKENS
-#define GG_L2_TOKENS 1
+#define GG_L2_TOKENS 0
 #endif
 #ifndef GG_L2_WEIGHTS
 #define GG_L2_WEIGHTS 2
@@ -72,6 +73,11 @@ constexpr int NUM_THREADS = 32 * (FIX_WARP + 1);
 // completes. It also bounds how late an aborting role notices the abort flag.
 #ifndef GG_WAIT_SLICE_NS
 #define GG_WAIT_SLICE_NS 200000
+#endif
+// Every other tile a CTA processes walks its reduction backwards, so that the operand
+// slabs a wave reads last are the first the next wave needs (they are still in L2).
+#ifndef GG_SERPENTINE
+#define GG_SERPENTINE 1
 #endif
 // Back-off (ns) of the epilogue warps while they wait for an accumulator (0 = spin).
 #ifndef GG_EPI_BACKOFF_NS
@@ -435,9 +441,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     bool ok = true;
     const int32_t row_off = (int32_t)rank * BM;         // this CTA's rows of a pair tile
     const int32_t col_off = (int32_t)rank * L::B_COLS;  // this CTA's columns of B
-    for (int32_t t = unit0; t < total && ok; t += units) {
+    for (int32_t t = unit0, it = 0; t < total && ok; t += units, ++it) {
       const Tile tl = decode_tile<MODE, BN, TM>(t, p, sh);
-      for (int32_t kb = 0; kb < tl.kblocks; ++kb) {
+      const bool rev = GG_SERPENTINE && (it & 1);
+      for (int32_t kq = 0; kq < tl.kblocks; ++kq) {
+        const int32_t kb = rev ? tl.kblocks - 1 - kq : kq;  // reduction block of this stage
         if (!warp_wait(&sh.empty[stage], phase ^ 1u, sh, p, false)) { ok = false; break; }
         uint8_t* sA = smem + L::OFF_A + stage * L::A_BYTES;
         uint8_t* sB = smem + L::OFF_B + stage * L::B_BYTES;
@@ -581,9 +589,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t stage = 0, phase = 0, acc_iter = 0;
       uint32_t fixed_par = 0;  // per stage: next phase of fixed[] (pair wgrad)
       bool ok = true;
-      for (int32_t t = unit0; t < total && ok; t += units) {
+      for (int32_t t = unit0, it = 0; t < total && ok; t += units, ++it) {
         const Tile tl = decode_tile<MODE, BN, TM>(t, p, sh);
         if (tl.kblocks == 0) continue;  // Wgrad of an empty expert: the epilogue writes zeros
+        const bool rev = GG_SERPENTINE && (it & 1);
         const uint32_t a = acc_iter & 1u;
         if (!wait_bounded(&sh.tempty[a], ((acc_iter >> 1) & 1u) ^ 1u, sh, p, true, PAIR)) {
           ok = false;
@@ -591,7 +600,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + a * BN;
-        for (int32_t kb = 0; kb < tl.kblocks; ++kb) {
+        for (int32_t kq = 0; kq < tl.kblocks; ++kq) {
+          const int32_t kb = rev ? tl.kblocks - 1 - kq : kq;
           if (!wait_bounded(&sh.full[stage], phase, sh, p, true)) { ok = false; break; }
 #if GG_FENCE_PER_STAGE
           ptx::tc_fence_after();
@@ -616,7 +626,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int k = 0; k < BK / UMMA_K; ++k) {
             if (k < nsub) {
-              const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+              const uint32_t acc = (kq > 0 || k > 0) ? 1u : 0u;  // the first stage overwrites
               if constexpr (PAIR)
                 ptx::mma_bf16_pair(d_tmem, adesc + k * A_STEP, bdesc + k * B_STEP, IDESC, acc);
               else
@@ -732,10 +742,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // operands so that they add nothing (the MMA reads no row past ceil16(rem)); a token row
     // is one 128-byte line of every 64-wide chunk.
     uint32_t stage = 0, landed_par = 0;
-    for (int32_t t = unit0; t < total; t += units) {
+    for (int32_t t = unit0, it = 0; t < total; t += units, ++it) {
       const Tile tl = decode_tile<MODE, BN, TM>(t, p, sh);
+      const bool rev = GG_SERPENTINE && (it & 1);
       bool ok = true;
-      for (int32_t kb = 0; kb < tl.kblocks; ++kb) {
+      for (int32_t kq = 0; kq < tl.kblocks; ++kq) {
+        const int32_t kb = rev ? tl.kblocks - 1 - kq : kq;
         const int32_t rem = tl.tok_len - kb * BK;
         if (rem < BK) {
           const uint32_t lp = (landed_par >> stage) & 1u;
