@@ -100,6 +100,11 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
             out, _ = self.proc.communicate()
+        return self.parse(out)
+
+    @staticmethod
+    def parse(out: str):
+        """Summary of `nvidia-smi --format=csv,noheader,nounits` lines of FIELDS."""
         rows = []
         for line in out.strip().splitlines():
             parts = [x.strip() for x in line.split(",")]
@@ -115,6 +120,15 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(loaded) if loaded else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
                 "samples": len(rows)}
+
+
+def reduce_max(value: float, device) -> float:
+    """Max of `value` over all ranks (identity without a process group)."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
 
 
 def dist_env():
@@ -271,10 +285,7 @@ def run_ours(args):
     total_ms = t_start.elapsed_time(t_end)
     per_pass_ms = [sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
                    / args.steps for j in range(4)]
-    if ws > 1:
-        t = torch.tensor([total_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = reduce_max(total_ms, dev)
     ms_per_step = total_ms / args.steps
     value = ws * step_flops / (ms_per_step * 1e-3) / 1e12
 
@@ -383,11 +394,7 @@ def run_e2e(args, gg, r, m, dev, stream, ws, barrier):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    ms = e0.elapsed_time(e1) / steps
-    if ws > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = reduce_max(e0.elapsed_time(e1) / steps, dev)
     flops = 3 * r.flops + m.flops
     return {"value": ws * flops / (ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms,
             "steps": steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
