@@ -240,6 +240,7 @@ int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 constexpr int kBN = 256;
 constexpr int kStages = 4;      // single CTA: 48 KB per stage
 constexpr int kPairStages = 6;  // CTA pair: 32 KB per stage and CTA
+constexpr int kMaskedBN = 128;  // masked forward: 128 x 128 tiles, 32 KB per stage
 
 // CTA pairs halve the operand traffic per SM but quantise groups to 256-row tiles; they pay
 // off once the average group is long.
@@ -365,10 +366,14 @@ gg_status gg_masked_forward(const void* A, const void* W, const int32_t* masked_
   if (mmax == 0) return GG_OK;
   if (A == nullptr || out == nullptr) return GG_ERR_INVALID_ARG;
   if (!aligned16(A) || !aligned16(W) || !aligned16(out)) return GG_ERR_UNSUPPORTED;
+  // A handful of experts with at most mmax rows each: narrower N-tiles spread the weight
+  // reads (the whole cost of this memory-bound shape) over more SMs, and A is fetched in
+  // 32-row boxes covering only the active rows.
   const bool chunked = (N % 64) == 0;
   CUtensorMap ma, mb;
-  if (!map_2d(&ma, A, (int64_t)E * mmax, K, 64, gg::BM)) return GG_ERR_CUDA;
-  if (chunked ? !map_w_chunked(&mb, W, E, K, N, 64, kBN / 64) : !map_w(&mb, W, E, K, N, 64, 64))
+  if (!map_2d(&ma, A, (int64_t)E * mmax, K, 64, 32)) return GG_ERR_CUDA;
+  if (chunked ? !map_w_chunked(&mb, W, E, K, N, 64, kMaskedBN / 64)
+              : !map_w(&mb, W, E, K, N, 64, 64))
     return GG_ERR_CUDA;
   gg::Params p = base_params(masked_m, out, dev_status, (int64_t)E * mmax, E);
   p.b_chunked = chunked ? 1 : 0;
@@ -376,8 +381,8 @@ gg_status gg_masked_forward(const void* A, const void* W, const int32_t* masked_
   p.red_len = (int32_t)K;
   p.out_cols = (int32_t)N;
   set_store_width(&p, out, N);
-  const int64_t tiles = (int64_t)E * cdiv(mmax, gg::BM) * cdiv(N, kBN);
-  return launch<Mode::Masked, kBN, kStages, false>(ma, mb, p, tiles, di, stream);
+  const int64_t tiles = (int64_t)E * cdiv(mmax, gg::BM) * cdiv(N, kMaskedBN);
+  return launch<Mode::Masked, kMaskedBN, kPairStages, false>(ma, mb, p, tiles, di, stream);
 }
 
 const char* gg_status_string(gg_status s) {

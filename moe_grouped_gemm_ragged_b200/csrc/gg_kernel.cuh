@@ -523,9 +523,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           } else {
             // a wgrad tail stage lands on landed[] first; full[] completes after the fix-up
             uint64_t* lb = tail ? &sh.landed[stage] : fb;
-            ptx::mbar_arrive_expect_tx(lb, L::STAGE_BYTES);
+            if constexpr (MODE == Mode::Masked) {
+              // only the group's rows of A, in 32-row boxes; the MMA also reads the stale
+              // rows after them, which only reach accumulator rows that are never stored
+              int64_t valid = tl.row_end - (int64_t)tl.a_row0;
+              if (valid > BM) valid = BM;
+              const int32_t nbox = (int32_t)((valid + 31) / 32);
+              ptx::mbar_arrive_expect_tx(lb, (uint32_t)nbox * 32u * 128u + L::B_BYTES);
+              for (int32_t b = 0; b < nbox; ++b)
+                ptx::tma_load_2d(sA + b * 4096, &mapA, lb, kb * BK, tl.a_row0 + b * 32, pol_tok);
+            } else {
+              ptx::mbar_arrive_expect_tx(lb, L::STAGE_BYTES);
+            }
             if constexpr (MODE == Mode::Forward || MODE == Mode::Masked) {
-              ptx::tma_load_2d(sA, &mapA, lb, kb * BK, tl.a_row0, pol_tok);
+              if constexpr (MODE == Mode::Forward)
+                ptx::tma_load_2d(sA, &mapA, lb, kb * BK, tl.a_row0, pol_tok);
               if (p.b_chunked) {
                 ptx::tma_load_4d(sB, &mapB, lb, 0, kb * BK, tl.n0 / 64, tl.e, pol_w);
               } else {

@@ -169,3 +169,22 @@ def test_repeat_calls_bit_identical(variant):
     b = run_ragged(r)
     for x, y in zip(a[:3], b[:3]):
         assert bool((x.view(torch.int16) == y.view(torch.int16)).all())
+
+
+@pytest.mark.parametrize("N", [2048, 264])
+def test_masked_counts_across_box_and_tile_edges(N):
+    """mmax=256 (two row tiles per expert), counts around the 32-row A boxes and the 128-row
+    tiles, N with and without 64-wide chunks; inactive rows NaN and untouched."""
+    counts = [0, 1, 31, 32, 33, 127, 128, 129, 255, 256]
+    m = workloads.make_masked(E=len(counts), mmax=256, K=192, N=N, masked_m=counts, seed=61)
+    out = sentinel((m.E, m.mmax, m.N))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    gg.masked_forward(m.A.cuda(), m.W.cuda(), torch.from_numpy(m.masked_m).cuda(), out,
+                      status=st)
+    torch.cuda.synchronize()
+    s = int(st.item())
+    assert s & gg.DEV_LAUNCHED and (s & gg.DEV_ERROR_MASK) == 0
+    ref, act, _ = oracle.masked_forward(m.A, m.W, m.masked_m)
+    flat = out.view(-1, m.N)
+    assert_close(to_f64(flat[torch.from_numpy(np.nonzero(act)[0]).cuda()]), ref[act], "masked")
+    assert bool(is_sentinel(flat[torch.from_numpy(np.nonzero(~act)[0]).cuda()]).all())
