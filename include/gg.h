@@ -114,6 +114,21 @@ GG_API gg_status gg_wgrad(const void* A, const void* dY, const int32_t* offs, vo
                    int32_t* dev_status, cudaStream_t stream);
 
 /*
+ * Wgrad into an fp32 buffer with scaling and accumulation (the main-grad update):
+ *   dW[e, k, n] = alpha * sum over rows r of group e of A[r, k] * dY[r, n]
+ *                 + beta * dW[e, k, n]
+ *   A bf16 [rows_alloc, K]; dY bf16 [rows_alloc, N]; dW fp32 [E, K, N], read (only when
+ *   beta != 0) and written in full, in place; an empty group gives beta * dW (0 when
+ *   beta == 0). The product is accumulated in fp32 and added without a bf16 rounding.
+ * Passage: TransformerEngine PR 3542, "Changes" (FP32 outputs, fused accumulation and
+ * explicit alpha/beta; a rounded BF16 product added separately would not keep the fused
+ * accumulation's precision).
+ */
+GG_API gg_status gg_wgrad_f32(const void* A, const void* dY, const int32_t* offs, float* dW,
+                              float alpha, float beta, int64_t rows_alloc, int64_t K,
+                              int64_t N, int32_t E, int32_t* dev_status, cudaStream_t stream);
+
+/*
  * Masked forward: out[e, r, n] = sum_k A[e, r, k] * W[e, k, n] for r < masked_m[e].
  *   A bf16 [E, mmax, K]; W bf16 [E, K, N]; masked_m int32 [E], device;
  *   out bf16 [E, mmax, N]: rows r >= masked_m[e] untouched.

@@ -56,6 +56,9 @@ def lib() -> ctypes.CDLL:
         fn = getattr(L, name)
         fn.argtypes = sig
         fn.restype = ctypes.c_int
+    L.gg_wgrad_f32.argtypes = [P, P, P, P, ctypes.c_float, ctypes.c_float, i64, i64, i64, i32,
+                               P, P]
+    L.gg_wgrad_f32.restype = ctypes.c_int
     L.gg_status_string.argtypes = [ctypes.c_int]
     L.gg_status_string.restype = ctypes.c_char_p
     L.gg_set_watchdog_ns.argtypes = [ctypes.c_uint64]
@@ -187,6 +190,28 @@ def wgrad(A: torch.Tensor, dY: torch.Tensor, offs: torch.Tensor, dW: torch.Tenso
     return dW
 
 
+def wgrad_f32(A: torch.Tensor, dY: torch.Tensor, offs: torch.Tensor, dW: torch.Tensor, *,
+              alpha: float = 1.0, beta: float = 1.0, status: Optional[torch.Tensor] = None,
+              stream=None) -> torch.Tensor:
+    """dW[e] = alpha * A[rows of e]^T @ dY[rows of e] + beta * dW[e], fp32 dW updated in place
+    (beta=1 accumulates into a main-grad buffer; beta=0 overwrites without reading dW).
+
+    A bf16 [rows, K], dY bf16 [rows, N], offs int32 [E], dW float32 [E, K, N]."""
+    _check(A, "A", torch.bfloat16, 2)
+    _check(dY, "dY", torch.bfloat16, 2)
+    _check(offs, "offs", torch.int32, 1)
+    _check(dW, "dW", torch.float32, 3)
+    rows, K = A.shape
+    rows2, N = dY.shape
+    E = offs.numel()
+    if rows2 != rows or tuple(dW.shape) != (E, K, N):
+        raise ValueError("shape mismatch: A[rows,K], dY[rows,N], offs[E], dW[E,K,N]")
+    rc = lib().gg_wgrad_f32(_ptr(A), _ptr(dY), _ptr(offs), _ptr(dW), float(alpha), float(beta),
+                            rows, K, N, E, _status_ptr(status), _stream_handle(stream))
+    _raise(rc, "gg_wgrad_f32")
+    return dW
+
+
 def masked_forward(A: torch.Tensor, W: torch.Tensor, masked_m: torch.Tensor,
                    out: torch.Tensor, *, status: Optional[torch.Tensor] = None,
                    stream=None) -> torch.Tensor:
@@ -216,7 +241,7 @@ def grouped_mm(A: torch.Tensor, W: torch.Tensor, offs: torch.Tensor,
 
 
 __all__ = [
-    "forward", "dgrad", "wgrad", "masked_forward", "grouped_mm", "status_string", "version",
+    "forward", "dgrad", "wgrad", "wgrad_f32", "masked_forward", "grouped_mm", "status_string", "version",
     "set_watchdog_ns", "testing_skip_first_load", "testing_force_variant", "lib", "GGError", "LIB_PATH",
     "DEV_BAD_OFFSETS", "DEV_BAD_MASKED_M", "DEV_TIMEOUT", "DEV_ERROR_MASK", "DEV_LAUNCHED",
     "MAX_EXPERTS",

@@ -137,10 +137,10 @@ bool map_w(CUtensorMap* m, const void* W, int64_t E, int64_t K, int64_t N, uint3
   return make_map(m, W, 3, dims, str, box);
 }
 
-template <Mode MODE, int BN, int STAGES, bool PAIR>
+template <Mode MODE, int BN, int STAGES, bool PAIR, bool F32 = false>
 gg_status launch(const CUtensorMap& a, const CUtensorMap& b, const gg::Params& p,
                  int64_t tiles_upper, const DeviceInfo& di, cudaStream_t stream) {
-  auto kern = gg::grouped_gemm_kernel<MODE, BN, STAGES, PAIR>;
+  auto kern = gg::grouped_gemm_kernel<MODE, BN, STAGES, PAIR, F32>;
   using L = gg::Layout<BN, STAGES, PAIR>;
   const size_t smem = L::bytes(p.E);
   int dev = 0;
@@ -251,6 +251,53 @@ bool use_pair(int64_t rows, int32_t E) {
   return rows >= 512 * (int64_t)E;
 }
 
+gg_status wgrad_impl(const void* A, const void* dY, const int32_t* offs, void* dW, bool f32,
+                     float alpha, float beta, int64_t rows_alloc, int64_t K, int64_t N,
+                     int32_t E, int32_t* dev_status, cudaStream_t stream) {
+  DeviceInfo di;
+  gg_status s = check_common(rows_alloc, K, N, E, offs, dev_status, &di);
+  if (s != GG_OK) return s;
+  if (dW == nullptr) return GG_ERR_INVALID_ARG;
+  if (!aligned16(dW)) return GG_ERR_UNSUPPORTED;
+  if (rows_alloc > 0) {
+    if (A == nullptr || dY == nullptr) return GG_ERR_INVALID_ARG;
+    if (!aligned16(A) || !aligned16(dY)) return GG_ERR_UNSUPPORTED;
+  } else {
+    // every group is empty: the maps are never used; dW only gets zeros (or beta * dW)
+    A = dW;
+    dY = dW;
+  }
+  const bool a_chunked = (K % 64) == 0, b_chunked = (N % 64) == 0;
+  // wgrad stays on single CTAs unless forced: measured faster on long groups (large shape
+  // 1159 vs 909 TFLOP/s) and equal on short ones
+  const bool pair = g_force_variant.load() == 2;
+  const uint32_t bcols = pair ? kBN / 2 : kBN;  // dY columns one CTA loads per stage
+  CUtensorMap ma, mb;
+  if (a_chunked ? !map_2d_chunked(&ma, A, rows_alloc, K, 64, gg::BM / 64)
+                : !map_2d(&ma, A, rows_alloc, K, 64, 64))
+    return GG_ERR_CUDA;
+  if (b_chunked ? !map_2d_chunked(&mb, dY, rows_alloc, N, 64, bcols / 64)
+                : !map_2d(&mb, dY, rows_alloc, N, 64, 64))
+    return GG_ERR_CUDA;
+  gg::Params p = base_params(offs, f32 ? nullptr : dW, dev_status, rows_alloc, E);
+  p.out_cols = (int32_t)N;
+  p.wg_K = (int32_t)K;
+  p.a_chunked = a_chunked ? 1 : 0;
+  p.b_chunked = b_chunked ? 1 : 0;
+  p.out_f32 = f32 ? reinterpret_cast<float*>(dW) : nullptr;
+  p.alpha = alpha;
+  p.beta = beta;
+  set_store_width(&p, dW, N);
+  if (pair) {
+    const int64_t tiles = (int64_t)E * cdiv(K, 2 * gg::BM) * cdiv(N, kBN);
+    if (f32) return launch<Mode::Wgrad, kBN, kPairStages, true, true>(ma, mb, p, tiles, di, stream);
+    return launch<Mode::Wgrad, kBN, kPairStages, true>(ma, mb, p, tiles, di, stream);
+  }
+  const int64_t tiles = (int64_t)E * cdiv(K, gg::BM) * cdiv(N, kBN);
+  if (f32) return launch<Mode::Wgrad, kBN, kStages, false, true>(ma, mb, p, tiles, di, stream);
+  return launch<Mode::Wgrad, kBN, kStages, false>(ma, mb, p, tiles, di, stream);
+}
+
 }  // namespace
 
 extern "C" {
@@ -315,43 +362,14 @@ gg_status gg_dgrad(const void* dY, const void* W, const int32_t* offs, void* dX,
 gg_status gg_wgrad(const void* A, const void* dY, const int32_t* offs, void* dW,
                    int64_t rows_alloc, int64_t K, int64_t N, int32_t E, int32_t* dev_status,
                    cudaStream_t stream) {
-  DeviceInfo di;
-  gg_status s = check_common(rows_alloc, K, N, E, offs, dev_status, &di);
-  if (s != GG_OK) return s;
-  if (dW == nullptr) return GG_ERR_INVALID_ARG;
-  if (!aligned16(dW)) return GG_ERR_UNSUPPORTED;
-  if (rows_alloc > 0) {
-    if (A == nullptr || dY == nullptr) return GG_ERR_INVALID_ARG;
-    if (!aligned16(A) || !aligned16(dY)) return GG_ERR_UNSUPPORTED;
-  } else {
-    // every group is empty: the maps are never used; dW only gets zeros
-    A = dW;
-    dY = dW;
-  }
-  const bool a_chunked = (K % 64) == 0, b_chunked = (N % 64) == 0;
-  // wgrad stays on single CTAs unless forced: measured faster on long groups (large shape
-  // 1159 vs 909 TFLOP/s) and equal on short ones
-  const bool pair = g_force_variant.load() == 2;
-  const uint32_t bcols = pair ? kBN / 2 : kBN;  // dY columns one CTA loads per stage
-  CUtensorMap ma, mb;
-  if (a_chunked ? !map_2d_chunked(&ma, A, rows_alloc, K, 64, gg::BM / 64)
-                : !map_2d(&ma, A, rows_alloc, K, 64, 64))
-    return GG_ERR_CUDA;
-  if (b_chunked ? !map_2d_chunked(&mb, dY, rows_alloc, N, 64, bcols / 64)
-                : !map_2d(&mb, dY, rows_alloc, N, 64, 64))
-    return GG_ERR_CUDA;
-  gg::Params p = base_params(offs, dW, dev_status, rows_alloc, E);
-  p.out_cols = (int32_t)N;
-  p.wg_K = (int32_t)K;
-  set_store_width(&p, dW, N);
-  p.a_chunked = a_chunked ? 1 : 0;
-  p.b_chunked = b_chunked ? 1 : 0;
-  if (pair) {
-    const int64_t tiles = (int64_t)E * cdiv(K, 2 * gg::BM) * cdiv(N, kBN);
-    return launch<Mode::Wgrad, kBN, kPairStages, true>(ma, mb, p, tiles, di, stream);
-  }
-  const int64_t tiles = (int64_t)E * cdiv(K, gg::BM) * cdiv(N, kBN);
-  return launch<Mode::Wgrad, kBN, kStages, false>(ma, mb, p, tiles, di, stream);
+  return wgrad_impl(A, dY, offs, dW, false, 1.f, 0.f, rows_alloc, K, N, E, dev_status, stream);
+}
+
+gg_status gg_wgrad_f32(const void* A, const void* dY, const int32_t* offs, float* dW,
+                       float alpha, float beta, int64_t rows_alloc, int64_t K, int64_t N,
+                       int32_t E, int32_t* dev_status, cudaStream_t stream) {
+  return wgrad_impl(A, dY, offs, dW, true, alpha, beta, rows_alloc, K, N, E, dev_status,
+                    stream);
 }
 
 gg_status gg_masked_forward(const void* A, const void* W, const int32_t* masked_m, void* out,

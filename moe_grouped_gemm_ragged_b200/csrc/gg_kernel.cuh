@@ -107,6 +107,10 @@ struct Params {
   int32_t a_chunked;
   int32_t b_chunked;
   int32_t out_v8;          // 1 when every output row starts 32-byte aligned (256-bit stores)
+  // fp32 output with scaling and accumulation (out_f32 = alpha * product + beta * out_f32)
+  float* out_f32;
+  float alpha;
+  float beta;
 };
 
 template <int BN, int STAGES, bool PAIR>
@@ -339,7 +343,7 @@ __device__ __forceinline__ Tile decode_tile(int32_t t, const Params& p, const Sh
 }
 
 // ---------------------------------------------------------------- kernel
-template <Mode MODE, int BN, int STAGES, bool PAIR>
+template <Mode MODE, int BN, int STAGES, bool PAIR, bool F32 = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap mapA,
                         const __grid_constant__ CUtensorMap mapB, const Params p) {
@@ -693,10 +697,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int32_t col0 = tl.n0 + c_off;
       if (tl.kblocks == 0) {
         if (row_ok) {
-          for (int c = 0; c < CW; c += 8) {
-            const int32_t col = col0 + c;
-            if (col < p.out_cols)
-              *reinterpret_cast<uint4*>(orow_ptr + col) = make_uint4(0u, 0u, 0u, 0u);
+          if constexpr (F32) {
+            // the product is zero: out = beta * out (nothing is read when beta == 0)
+            float* orow_f = p.out_f32 + orow * (int64_t)p.out_cols;
+            for (int c = 0; c < CW; c += 4) {
+              const int32_t col = col0 + c;
+              if (col < p.out_cols) {
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (p.beta != 0.f) {
+                  const float4 o = *reinterpret_cast<const float4*>(orow_f + col);
+                  v = make_float4(p.beta * o.x, p.beta * o.y, p.beta * o.z, p.beta * o.w);
+                }
+                *reinterpret_cast<float4*>(orow_f + col) = v;
+              }
+            }
+          } else {
+            for (int c = 0; c < CW; c += 8) {
+              const int32_t col = col0 + c;
+              if (col < p.out_cols)
+                *reinterpret_cast<uint4*>(orow_ptr + col) = make_uint4(0u, 0u, 0u, 0u);
+            }
           }
         }
         continue;
@@ -714,7 +734,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t(&nxt)[32] = ((c / 32) & 1) ? r0 : r1;
         ptx::tmem_ld_wait();
         if (c + 32 < CW) ptx::tmem_ld_32x32b_x32(taddr + c + 32, nxt);
-        if (row_ok) {
+        if (F32 && row_ok) {
+          // fp32 out = alpha * acc + beta * out; the old value is read only when beta != 0
+          float* orow_f = p.out_f32 + orow * (int64_t)p.out_cols;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int32_t col = col0 + c + j * 4;
+            if (col < p.out_cols) {
+              float4 v = make_float4(p.alpha * __uint_as_float(cur[4 * j]),
+                                     p.alpha * __uint_as_float(cur[4 * j + 1]),
+                                     p.alpha * __uint_as_float(cur[4 * j + 2]),
+                                     p.alpha * __uint_as_float(cur[4 * j + 3]));
+              if (p.beta != 0.f) {
+                const float4 o = *reinterpret_cast<const float4*>(orow_f + col);
+                v.x = fmaf(p.beta, o.x, v.x);
+                v.y = fmaf(p.beta, o.y, v.y);
+                v.z = fmaf(p.beta, o.z, v.z);
+                v.w = fmaf(p.beta, o.w, v.w);
+              }
+              *reinterpret_cast<float4*>(orow_f + col) = v;
+            }
+          }
+        } else if (row_ok) {
           uint32_t packed[16];
 #pragma unroll
           for (int h = 0; h < 16; ++h) {

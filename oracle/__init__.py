@@ -157,6 +157,21 @@ def wgrad(A, dY, offs, E=None, ks=None, threads=None):
     return out
 
 
+def wgrad_accumulate(A, dY, offs, old, alpha: float, beta: float, ks=None, threads=None):
+    """fp64 reference of the fp32 wgrad with scaling and accumulation:
+    dW[e, k, n] = alpha * sum_{r in group e} A[r,k] dY[r,n] + beta * old[e, k, n]
+    (TransformerEngine PR 3542, "Changes": FP32 outputs, fused accumulation, explicit
+    alpha/beta). ``old`` is the fp32 buffer before the call ([E, K, N]); with beta == 0 it
+    is not read (so NaN there does not matter). Returns dW[E, len(ks), N]."""
+    prod = wgrad(A, dY, offs, ks=ks, threads=threads)
+    out = float(alpha) * prod
+    if beta != 0.0:
+        o = np.asarray(old, dtype=np.float32).astype(np.float64)
+        kk = np.arange(o.shape[1]) if ks is None else np.asarray(ks, dtype=np.int64)
+        out = out + float(beta) * o[:, kk, :]
+    return out
+
+
 def masked_forward(A, W, masked_m, rows=None, threads=None):
     """fp64 masked forward on flat rows e*mmax+r (default: all). Returns
     (out[nrows,N], active[nrows], bad)."""

@@ -188,3 +188,38 @@ def test_masked_counts_across_box_and_tile_edges(N):
     flat = out.view(-1, m.N)
     assert_close(to_f64(flat[torch.from_numpy(np.nonzero(act)[0]).cuda()]), ref[act], "masked")
     assert bool(is_sentinel(flat[torch.from_numpy(np.nonzero(~act)[0]).cuda()]).all())
+
+
+@pytest.mark.parametrize("alpha,beta", [(1.0, 0.0), (0.5, 1.0), (-2.0, 0.25)])
+def test_wgrad_f32_scaling_and_accumulation(alpha, beta, variant):
+    """fp32 dW = alpha * A_e^T dY_e + beta * dW in place; beta == 0 never reads dW (NaN there
+    stays out of the result); an empty expert gives beta * dW."""
+    r = workloads.make_ragged_custom(len(SWEEP), 200, 328, SWEEP, seed=73, tail=64)
+    A, dY = r.A.cuda(), r.dY.cuda()
+    offs = torch.from_numpy(r.offs).cuda()
+    rng = np.random.default_rng(3)
+    old = rng.standard_normal((r.E, r.K, r.N)).astype(np.float32) * 10
+    if beta == 0.0:
+        old[:] = np.nan
+    dW = torch.from_numpy(old.copy()).cuda()
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    gg.wgrad_f32(A, dY, offs, dW, alpha=alpha, beta=beta, status=st)
+    torch.cuda.synchronize()
+    s = int(st.item())
+    assert s & gg.DEV_LAUNCHED and (s & gg.DEV_ERROR_MASK) == 0
+    ref = oracle.wgrad_accumulate(r.A, r.dY, r.offs, old, alpha, beta)
+    assert_close(dW.double().cpu().numpy(), ref, "wgrad_f32")
+
+
+def test_wgrad_f32_accumulates_over_two_calls():
+    """Two accumulating calls into one main-grad buffer equal the sum of two products."""
+    r = workloads.make_ragged("gateup", tail=128, device="cuda")
+    offs = torch.from_numpy(r.offs).cuda()
+    dW = torch.zeros(r.E, r.K, r.N, dtype=torch.float32, device="cuda")
+    gg.wgrad_f32(r.A, r.dY, offs, dW, alpha=1.0, beta=1.0)
+    gg.wgrad_f32(r.A, r.dY, offs, dW, alpha=1.0, beta=1.0)
+    torch.cuda.synchronize()
+    ks = sample_k(r.K, 5)
+    ref = 2.0 * oracle.wgrad(oracle.as_u16(r.A), oracle.as_u16(r.dY), r.offs, ks=ks)
+    got = dW[:, torch.from_numpy(ks).cuda(), :].double().cpu().numpy()
+    assert_close(got, ref, "wgrad_f32 accumulated twice")

@@ -309,3 +309,24 @@ def test_round_bf16_matches_torch_on_float_values_and_ties():
     assert oracle.round_bf16([1 + 2 ** -8])[0] == 0x3F80
     assert oracle.round_bf16([1 + 3 * 2 ** -8])[0] == 0x3F82
     assert oracle.round_bf16([1 + 2 ** -8 + 2 ** -40])[0] == 0x3F81
+
+
+def test_wgrad_accumulate_reduces_and_is_exact_on_integers():
+    """The fp32 accumulating wgrad: alpha=1,beta=0 is plain wgrad; alpha=0 leaves beta*old;
+    small integers give exact values; NaN in `old` is ignored when beta == 0."""
+    sizes = [5, 0, 9]
+    r = workloads.make_ragged_custom(3, 16, 24, sizes, seed=71, tail=2)
+    old = np.random.default_rng(1).standard_normal((3, 16, 24)).astype(np.float32)
+    base = oracle.wgrad(r.A, r.dY, r.offs)
+    np.testing.assert_array_equal(oracle.wgrad_accumulate(r.A, r.dY, r.offs, old, 1.0, 0.0), base)
+    np.testing.assert_array_equal(oracle.wgrad_accumulate(r.A, r.dY, r.offs, old, 0.0, 2.0),
+                                  2.0 * old.astype(np.float64))
+    nan_old = np.full((3, 16, 24), np.nan, np.float32)
+    assert np.all(np.isfinite(oracle.wgrad_accumulate(r.A, r.dY, r.offs, nan_old, 0.5, 0.0)))
+    # integer probe: A = 1, dY = 2 on group rows; old = 3 -> dW = alpha*2*m_e + beta*3
+    A = torch.ones(16, 4, dtype=torch.bfloat16)
+    dY = torch.full((16, 8), 2.0, dtype=torch.bfloat16)
+    offs = np.array([5, 5, 14], np.int32)
+    got = oracle.wgrad_accumulate(A, dY, offs, np.full((3, 4, 8), 3.0, np.float32), 0.5, -1.0)
+    for e, m in enumerate([5, 0, 9]):
+        assert np.all(got[e] == 0.5 * 2 * m - 3.0)
