@@ -140,6 +140,40 @@ GG_API gg_status gg_masked_forward(const void* A, const void* W, const int32_t* 
                             void* out, int64_t mmax, int64_t K, int64_t N, int32_t E,
                             int32_t* dev_status, cudaStream_t stream);
 
+/* Forward epilogue fused into gg_forward_ex / gg_masked_forward_ex.
+ *   h[r, n] = sum_k A[r, k] * W[e, k, n] + s[r] * bias[e, n]
+ *     bias        bf16 [E, N], 16-byte aligned, or NULL (no bias)
+ *     bias_scale  fp32, indexed by output row (the flat row e*mmax + r in the masked layout);
+ *                 read only for rows inside a group, i.e. the logical tokens, never for the
+ *                 unused capacity; NULL means s = 1. Ignored when bias is NULL.
+ *   act GG_ACT_NONE:     out[r, n] = h[r, n]                      (out has N columns)
+ *   act GG_ACT_SILU_MUL: gate and up columns interleaved in blocks of 128 inside every block
+ *                        of 256 columns (N % 256 == 0, else GG_ERR_UNSUPPORTED):
+ *                        out[r, 128 b + i] = silu(h[r, 256 b + i]) * h[r, 256 b + 128 + i],
+ *                        silu(x) = x / (1 + e^-x)                 (out has N / 2 columns)
+ * Passages: TransformerEngine PR 3542 review ("Expand per-group bias across result capacity",
+ * "Per-token bias scale", scaling limited to the logical rows); sglang PR 32385, "Cause"
+ * (SiLU-and-mul between the gate-up and the down GEMM, written only for active rows). */
+#define GG_ACT_NONE 0
+#define GG_ACT_SILU_MUL 1
+typedef struct gg_epilogue {
+  const void* bias;
+  const float* bias_scale;
+  int32_t act;
+} gg_epilogue;
+
+/* gg_forward with a fused epilogue (epi may be NULL: same as gg_forward). out is
+   bf16 [rows_alloc, N] (GG_ACT_NONE) or [rows_alloc, N/2] (GG_ACT_SILU_MUL). */
+GG_API gg_status gg_forward_ex(const void* A, const void* W, const int32_t* offs, void* out,
+                               int64_t rows_alloc, int64_t K, int64_t N, int32_t E,
+                               const gg_epilogue* epi, int32_t* dev_status, cudaStream_t stream);
+
+/* gg_masked_forward with a fused epilogue; out is [E, mmax, N] or [E, mmax, N/2]. */
+GG_API gg_status gg_masked_forward_ex(const void* A, const void* W, const int32_t* masked_m,
+                                      void* out, int64_t mmax, int64_t K, int64_t N, int32_t E,
+                                      const gg_epilogue* epi, int32_t* dev_status,
+                                      cudaStream_t stream);
+
 /* A static, human-readable name for a status. */
 GG_API const char* gg_status_string(gg_status s);
 

@@ -31,6 +31,13 @@ MAX_EXPERTS = 1024
 
 _lib = None
 
+ACT_NONE, ACT_SILU_MUL = 0, 1
+
+
+class _Epilogue(ctypes.Structure):
+    _fields_ = [("bias", ctypes.c_void_p), ("bias_scale", ctypes.c_void_p),
+                ("act", ctypes.c_int32)]
+
 
 class GGError(RuntimeError):
     """A non-OK status returned by the C ABI."""
@@ -59,6 +66,11 @@ def lib() -> ctypes.CDLL:
     L.gg_wgrad_f32.argtypes = [P, P, P, P, ctypes.c_float, ctypes.c_float, i64, i64, i64, i32,
                                P, P]
     L.gg_wgrad_f32.restype = ctypes.c_int
+    L.gg_forward_ex.argtypes = [P, P, P, P, i64, i64, i64, i32, ctypes.POINTER(_Epilogue), P, P]
+    L.gg_forward_ex.restype = ctypes.c_int
+    L.gg_masked_forward_ex.argtypes = [P, P, P, P, i64, i64, i64, i32,
+                                       ctypes.POINTER(_Epilogue), P, P]
+    L.gg_masked_forward_ex.restype = ctypes.c_int
     L.gg_status_string.argtypes = [ctypes.c_int]
     L.gg_status_string.restype = ctypes.c_char_p
     L.gg_set_watchdog_ns.argtypes = [ctypes.c_uint64]
@@ -148,6 +160,64 @@ def forward(A: torch.Tensor, W: torch.Tensor, offs: torch.Tensor, out: torch.Ten
     rc = lib().gg_forward(_ptr(A), _ptr(W), _ptr(offs), _ptr(out), rows, K, N, E,
                           _status_ptr(status), _stream_handle(stream))
     _raise(rc, "gg_forward")
+    return out
+
+
+def _epilogue(bias, bias_scale, act, E, N):
+    if bias is not None:
+        _check(bias, "bias", torch.bfloat16, 2)
+        if tuple(bias.shape) != (E, N):
+            raise ValueError("bias must be [E, N]")
+    if bias_scale is not None:
+        _check(bias_scale, "bias_scale", torch.float32, 1)
+    if act not in (ACT_NONE, ACT_SILU_MUL):
+        raise ValueError("act must be ACT_NONE or ACT_SILU_MUL")
+    return _Epilogue(_ptr(bias), _ptr(bias_scale), act)
+
+
+def forward_ex(A: torch.Tensor, W: torch.Tensor, offs: torch.Tensor, out: torch.Tensor, *,
+               bias: Optional[torch.Tensor] = None, bias_scale: Optional[torch.Tensor] = None,
+               act: int = ACT_NONE, status: Optional[torch.Tensor] = None,
+               stream=None) -> torch.Tensor:
+    """Forward with a fused epilogue: h = A @ W[e] + bias_scale[r] * bias[e]; with
+    act=ACT_SILU_MUL out = silu(gate) * up over gate/up column blocks of 128 (N % 256 == 0),
+    and out has N/2 columns. bias_scale is read only for rows inside a group."""
+    _check(A, "A", torch.bfloat16, 2)
+    _check(W, "W", torch.bfloat16, 3)
+    _check(offs, "offs", torch.int32, 1)
+    _check(out, "out", torch.bfloat16, 2)
+    rows, K = A.shape
+    E, K2, N = W.shape
+    ncols = N // 2 if act == ACT_SILU_MUL else N
+    if K2 != K or offs.numel() != E or tuple(out.shape) != (rows, ncols):
+        raise ValueError("shape mismatch: A[rows,K], W[E,K,N], offs[E], out[rows,N or N/2]")
+    epi = _epilogue(bias, bias_scale, act, E, N)
+    rc = lib().gg_forward_ex(_ptr(A), _ptr(W), _ptr(offs), _ptr(out), rows, K, N, E,
+                             ctypes.byref(epi), _status_ptr(status), _stream_handle(stream))
+    _raise(rc, "gg_forward_ex")
+    return out
+
+
+def masked_forward_ex(A: torch.Tensor, W: torch.Tensor, masked_m: torch.Tensor,
+                      out: torch.Tensor, *, bias: Optional[torch.Tensor] = None,
+                      bias_scale: Optional[torch.Tensor] = None, act: int = ACT_NONE,
+                      status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Masked forward with the fused epilogue of forward_ex; bias_scale is indexed by the
+    flat row e*mmax + r; out is [E, mmax, N] or [E, mmax, N/2]."""
+    _check(A, "A", torch.bfloat16, 3)
+    _check(W, "W", torch.bfloat16, 3)
+    _check(masked_m, "masked_m", torch.int32, 1)
+    _check(out, "out", torch.bfloat16, 3)
+    E, mmax, K = A.shape
+    E2, K2, N = W.shape
+    ncols = N // 2 if act == ACT_SILU_MUL else N
+    if E2 != E or K2 != K or masked_m.numel() != E or tuple(out.shape) != (E, mmax, ncols):
+        raise ValueError("shape mismatch: A[E,mmax,K], W[E,K,N], masked_m[E], out")
+    epi = _epilogue(bias, bias_scale, act, E, N)
+    rc = lib().gg_masked_forward_ex(_ptr(A), _ptr(W), _ptr(masked_m), _ptr(out), mmax, K, N, E,
+                                    ctypes.byref(epi), _status_ptr(status),
+                                    _stream_handle(stream))
+    _raise(rc, "gg_masked_forward_ex")
     return out
 
 
@@ -241,7 +311,8 @@ def grouped_mm(A: torch.Tensor, W: torch.Tensor, offs: torch.Tensor,
 
 
 __all__ = [
-    "forward", "dgrad", "wgrad", "wgrad_f32", "masked_forward", "grouped_mm", "status_string", "version",
+    "forward", "forward_ex", "dgrad", "wgrad", "wgrad_f32", "masked_forward",
+    "masked_forward_ex", "ACT_NONE", "ACT_SILU_MUL", "grouped_mm", "status_string", "version",
     "set_watchdog_ns", "testing_skip_first_load", "testing_force_variant", "lib", "GGError", "LIB_PATH",
     "DEV_BAD_OFFSETS", "DEV_BAD_MASKED_M", "DEV_TIMEOUT", "DEV_ERROR_MASK", "DEV_LAUNCHED",
     "MAX_EXPERTS",

@@ -137,10 +137,10 @@ bool map_w(CUtensorMap* m, const void* W, int64_t E, int64_t K, int64_t N, uint3
   return make_map(m, W, 3, dims, str, box);
 }
 
-template <Mode MODE, int BN, int STAGES, bool PAIR, bool F32 = false>
+template <Mode MODE, int BN, int STAGES, bool PAIR, bool F32 = false, int ACT = 0>
 gg_status launch(const CUtensorMap& a, const CUtensorMap& b, const gg::Params& p,
                  int64_t tiles_upper, const DeviceInfo& di, cudaStream_t stream) {
-  auto kern = gg::grouped_gemm_kernel<MODE, BN, STAGES, PAIR, F32>;
+  auto kern = gg::grouped_gemm_kernel<MODE, BN, STAGES, PAIR, F32, ACT>;
   using L = gg::Layout<BN, STAGES, PAIR>;
   const size_t smem = L::bytes(p.E);
   int dev = 0;
@@ -281,6 +281,7 @@ gg_status wgrad_impl(const void* A, const void* dY, const int32_t* offs, void* d
     return GG_ERR_CUDA;
   gg::Params p = base_params(offs, f32 ? nullptr : dW, dev_status, rows_alloc, E);
   p.out_cols = (int32_t)N;
+  p.prod_cols = (int32_t)N;
   p.wg_K = (int32_t)K;
   p.a_chunked = a_chunked ? 1 : 0;
   p.b_chunked = b_chunked ? 1 : 0;
@@ -298,13 +299,24 @@ gg_status wgrad_impl(const void* A, const void* dY, const int32_t* offs, void* d
   return launch<Mode::Wgrad, kBN, kStages, false>(ma, mb, p, tiles, di, stream);
 }
 
-}  // namespace
+// Checks the epilogue description and stores it in p. act SiLU-and-mul needs N % 256 == 0
+// (gate/up blocks of 128 columns inside every 256-column tile) and halves the output width.
+gg_status set_epilogue(gg::Params* p, const gg_epilogue* epi, int64_t N) {
+  p->bias_ld = (int32_t)N;
+  if (epi == nullptr) return GG_OK;
+  if (epi->act != GG_ACT_NONE && epi->act != GG_ACT_SILU_MUL) return GG_ERR_INVALID_ARG;
+  if (epi->bias != nullptr && !aligned16(epi->bias)) return GG_ERR_UNSUPPORTED;
+  if (epi->bias_scale != nullptr && (reinterpret_cast<uintptr_t>(epi->bias_scale) & 3u) != 0)
+    return GG_ERR_UNSUPPORTED;
+  if (epi->act == GG_ACT_SILU_MUL && (N % kBN) != 0) return GG_ERR_UNSUPPORTED;
+  p->bias = reinterpret_cast<const __nv_bfloat16*>(epi->bias);
+  p->bias_scale = epi->bias != nullptr ? epi->bias_scale : nullptr;
+  return GG_OK;
+}
 
-extern "C" {
-
-gg_status gg_forward(const void* A, const void* W, const int32_t* offs, void* out,
-                     int64_t rows_alloc, int64_t K, int64_t N, int32_t E, int32_t* dev_status,
-                     cudaStream_t stream) {
+gg_status forward_impl(const void* A, const void* W, const int32_t* offs, void* out,
+                       int64_t rows_alloc, int64_t K, int64_t N, int32_t E,
+                       const gg_epilogue* epi, int32_t* dev_status, cudaStream_t stream) {
   DeviceInfo di;
   gg_status s = check_common(rows_alloc, K, N, E, offs, dev_status, &di);
   if (s != GG_OK) return s;
@@ -312,6 +324,7 @@ gg_status gg_forward(const void* A, const void* W, const int32_t* offs, void* ou
   if (rows_alloc == 0) return GG_OK;  // no row can belong to a group
   if (A == nullptr || out == nullptr) return GG_ERR_INVALID_ARG;
   if (!aligned16(A) || !aligned16(W) || !aligned16(out)) return GG_ERR_UNSUPPORTED;
+  const bool silu = epi != nullptr && epi->act == GG_ACT_SILU_MUL;
   const bool pair = use_pair(rows_alloc, E);
   const bool chunked = (N % 64) == 0;
   const uint32_t bcols = pair ? kBN / 2 : kBN;
@@ -321,15 +334,87 @@ gg_status gg_forward(const void* A, const void* W, const int32_t* offs, void* ou
     return GG_ERR_CUDA;
   gg::Params p = base_params(offs, out, dev_status, rows_alloc, E);
   p.red_len = (int32_t)K;
-  p.out_cols = (int32_t)N;
   p.b_chunked = chunked ? 1 : 0;
-  set_store_width(&p, out, N);
+  if ((s = set_epilogue(&p, epi, N)) != GG_OK) return s;
+  const int64_t out_cols = silu ? N / 2 : N;
+  p.out_cols = (int32_t)out_cols;
+  p.prod_cols = (int32_t)N;
+  set_store_width(&p, out, out_cols);
   if (pair) {
     const int64_t tiles = (cdiv(rows_alloc, 2 * gg::BM) + E) * cdiv(N, kBN);
+    if (silu)
+      return launch<Mode::Forward, kBN, kPairStages, true, false, 1>(ma, mb, p, tiles, di, stream);
     return launch<Mode::Forward, kBN, kPairStages, true>(ma, mb, p, tiles, di, stream);
   }
   const int64_t tiles = (cdiv(rows_alloc, gg::BM) + E) * cdiv(N, kBN);
+  if (silu) return launch<Mode::Forward, kBN, kStages, false, false, 1>(ma, mb, p, tiles, di, stream);
   return launch<Mode::Forward, kBN, kStages, false>(ma, mb, p, tiles, di, stream);
+}
+
+gg_status masked_impl(const void* A, const void* W, const int32_t* masked_m, void* out,
+                      int64_t mmax, int64_t K, int64_t N, int32_t E, const gg_epilogue* epi,
+                      int32_t* dev_status, cudaStream_t stream) {
+  DeviceInfo di;
+  if (mmax < 0) return GG_ERR_INVALID_ARG;
+  if ((int64_t)E * mmax >= (int64_t(1) << 31)) return GG_ERR_UNSUPPORTED;
+  gg_status s = check_common((int64_t)E * mmax, K, N, E, masked_m, dev_status, &di);
+  if (s != GG_OK) return s;
+  if (W == nullptr) return GG_ERR_INVALID_ARG;
+  if (mmax == 0) return GG_OK;
+  if (A == nullptr || out == nullptr) return GG_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(W) || !aligned16(out)) return GG_ERR_UNSUPPORTED;
+  // A handful of experts with at most mmax rows each: narrower N-tiles spread the weight
+  // reads (the whole cost of this memory-bound shape) over more SMs, and A is fetched in
+  // 32-row boxes covering only the active rows. SiLU-and-mul needs gate and up columns in
+  // one tile, so it keeps 256-wide tiles.
+  const bool silu = epi != nullptr && epi->act == GG_ACT_SILU_MUL;
+  const int bn = silu ? kBN : kMaskedBN;
+  const bool chunked = (N % 64) == 0;
+  CUtensorMap ma, mb;
+  if (!map_2d(&ma, A, (int64_t)E * mmax, K, 64, 32)) return GG_ERR_CUDA;
+  if (chunked ? !map_w_chunked(&mb, W, E, K, N, 64, bn / 64) : !map_w(&mb, W, E, K, N, 64, 64))
+    return GG_ERR_CUDA;
+  gg::Params p = base_params(masked_m, out, dev_status, (int64_t)E * mmax, E);
+  p.b_chunked = chunked ? 1 : 0;
+  p.mmax = (int32_t)mmax;
+  p.red_len = (int32_t)K;
+  if ((s = set_epilogue(&p, epi, N)) != GG_OK) return s;
+  const int64_t out_cols = silu ? N / 2 : N;
+  p.out_cols = (int32_t)out_cols;
+  p.prod_cols = (int32_t)N;
+  set_store_width(&p, out, out_cols);
+  const int64_t tiles = (int64_t)E * cdiv(mmax, gg::BM) * cdiv(N, bn);
+  if (silu) return launch<Mode::Masked, kBN, kStages, false, false, 1>(ma, mb, p, tiles, di, stream);
+  return launch<Mode::Masked, kMaskedBN, kPairStages, false>(ma, mb, p, tiles, di, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+gg_status gg_forward(const void* A, const void* W, const int32_t* offs, void* out,
+                     int64_t rows_alloc, int64_t K, int64_t N, int32_t E, int32_t* dev_status,
+                     cudaStream_t stream) {
+  return forward_impl(A, W, offs, out, rows_alloc, K, N, E, nullptr, dev_status, stream);
+}
+
+gg_status gg_forward_ex(const void* A, const void* W, const int32_t* offs, void* out,
+                        int64_t rows_alloc, int64_t K, int64_t N, int32_t E,
+                        const gg_epilogue* epi, int32_t* dev_status, cudaStream_t stream) {
+  return forward_impl(A, W, offs, out, rows_alloc, K, N, E, epi, dev_status, stream);
+}
+
+gg_status gg_masked_forward(const void* A, const void* W, const int32_t* masked_m, void* out,
+                            int64_t mmax, int64_t K, int64_t N, int32_t E, int32_t* dev_status,
+                            cudaStream_t stream) {
+  return masked_impl(A, W, masked_m, out, mmax, K, N, E, nullptr, dev_status, stream);
+}
+
+gg_status gg_masked_forward_ex(const void* A, const void* W, const int32_t* masked_m, void* out,
+                               int64_t mmax, int64_t K, int64_t N, int32_t E,
+                               const gg_epilogue* epi, int32_t* dev_status,
+                               cudaStream_t stream) {
+  return masked_impl(A, W, masked_m, out, mmax, K, N, E, epi, dev_status, stream);
 }
 
 gg_status gg_dgrad(const void* dY, const void* W, const int32_t* offs, void* dX,
@@ -350,6 +435,7 @@ gg_status gg_dgrad(const void* dY, const void* W, const int32_t* offs, void* dX,
   gg::Params p = base_params(offs, dX, dev_status, rows_alloc, E);
   p.red_len = (int32_t)N;
   p.out_cols = (int32_t)K;
+  p.prod_cols = (int32_t)K;
   set_store_width(&p, dX, K);
   if (pair) {
     const int64_t tiles = (cdiv(rows_alloc, 2 * gg::BM) + E) * cdiv(K, kBN);
@@ -370,37 +456,6 @@ gg_status gg_wgrad_f32(const void* A, const void* dY, const int32_t* offs, float
                        int32_t E, int32_t* dev_status, cudaStream_t stream) {
   return wgrad_impl(A, dY, offs, dW, true, alpha, beta, rows_alloc, K, N, E, dev_status,
                     stream);
-}
-
-gg_status gg_masked_forward(const void* A, const void* W, const int32_t* masked_m, void* out,
-                            int64_t mmax, int64_t K, int64_t N, int32_t E, int32_t* dev_status,
-                            cudaStream_t stream) {
-  DeviceInfo di;
-  if (mmax < 0) return GG_ERR_INVALID_ARG;
-  if ((int64_t)E * mmax >= (int64_t(1) << 31)) return GG_ERR_UNSUPPORTED;
-  gg_status s = check_common((int64_t)E * mmax, K, N, E, masked_m, dev_status, &di);
-  if (s != GG_OK) return s;
-  if (W == nullptr) return GG_ERR_INVALID_ARG;
-  if (mmax == 0) return GG_OK;
-  if (A == nullptr || out == nullptr) return GG_ERR_INVALID_ARG;
-  if (!aligned16(A) || !aligned16(W) || !aligned16(out)) return GG_ERR_UNSUPPORTED;
-  // A handful of experts with at most mmax rows each: narrower N-tiles spread the weight
-  // reads (the whole cost of this memory-bound shape) over more SMs, and A is fetched in
-  // 32-row boxes covering only the active rows.
-  const bool chunked = (N % 64) == 0;
-  CUtensorMap ma, mb;
-  if (!map_2d(&ma, A, (int64_t)E * mmax, K, 64, 32)) return GG_ERR_CUDA;
-  if (chunked ? !map_w_chunked(&mb, W, E, K, N, 64, kMaskedBN / 64)
-              : !map_w(&mb, W, E, K, N, 64, 64))
-    return GG_ERR_CUDA;
-  gg::Params p = base_params(masked_m, out, dev_status, (int64_t)E * mmax, E);
-  p.b_chunked = chunked ? 1 : 0;
-  p.mmax = (int32_t)mmax;
-  p.red_len = (int32_t)K;
-  p.out_cols = (int32_t)N;
-  set_store_width(&p, out, N);
-  const int64_t tiles = (int64_t)E * cdiv(mmax, gg::BM) * cdiv(N, kMaskedBN);
-  return launch<Mode::Masked, kMaskedBN, kPairStages, false>(ma, mb, p, tiles, di, stream);
 }
 
 const char* gg_status_string(gg_status s) {

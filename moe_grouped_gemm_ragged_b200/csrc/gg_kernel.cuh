@@ -98,7 +98,9 @@ struct Params {
   int32_t E;
   int32_t mmax;            // masked mode only
   int32_t red_len;         // reduction length (Forward/Masked: K, Dgrad: N; Wgrad: unused)
-  int32_t out_cols;        // output columns (Forward/Masked/Wgrad: N, Dgrad: K)
+  int32_t out_cols;        // output columns (Forward/Masked/Wgrad: N, Dgrad: K; N/2 with
+                           // the SiLU-and-mul epilogue)
+  int32_t prod_cols;       // columns of the product the tiles cover (out_cols, or N)
   int32_t wg_K;            // Wgrad: K (rows of each dW[e])
   uint64_t watchdog_ns;
   int32_t debug_flags;     // bit 0: CTA 0 skips its first load (watchdog test)
@@ -111,6 +113,12 @@ struct Params {
   float* out_f32;
   float alpha;
   float beta;
+  // forward epilogue: h = product + s[row] * bias[e, col] (bf16 [E, N], may be null; s from
+  // bias_scale, fp32 indexed by output row, 1 when null); with SiLU-and-mul the output has
+  // N/2 columns (out_cols) and the product N (bias_ld)
+  const __nv_bfloat16* bias;
+  const float* bias_scale;
+  int32_t bias_ld;
 };
 
 template <int BN, int STAGES, bool PAIR>
@@ -216,7 +224,7 @@ template <Mode MODE, int BN, int TM>
 __device__ void build_table(const Params& p, const Shared& sh) {
   const uint32_t lane = ptx::lane_id();
   const int32_t E = p.E;
-  const int32_t NT = (p.out_cols + BN - 1) / BN;
+  const int32_t NT = (p.prod_cols + BN - 1) / BN;
   int64_t run_max = 0;   // running max of offsets seen so far (starts at t'_{-1} = 0)
   int32_t prev_end = 0;  // t'_{base-1}
   int32_t tiles_carry = 0;
@@ -300,7 +308,7 @@ __device__ void build_wgrad_order(const Params& p, const Shared& sh) {
 template <Mode MODE, int BN, int TM>
 __device__ __forceinline__ Tile decode_tile(int32_t t, const Params& p, const Shared& sh) {
   Tile tl;
-  const int32_t NT = (p.out_cols + BN - 1) / BN;
+  const int32_t NT = (p.prod_cols + BN - 1) / BN;
   if constexpr (MODE == Mode::Wgrad) {
     const int32_t KT = (p.wg_K + TM - 1) / TM;
     const int32_t per = KT * NT;
@@ -343,7 +351,8 @@ __device__ __forceinline__ Tile decode_tile(int32_t t, const Params& p, const Sh
 }
 
 // ---------------------------------------------------------------- kernel
-template <Mode MODE, int BN, int STAGES, bool PAIR, bool F32 = false>
+// ACT 1: SiLU-and-mul epilogue (gate and up columns interleaved in blocks of BN/2).
+template <Mode MODE, int BN, int STAGES, bool PAIR, bool F32 = false, int ACT = 0>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap mapA,
                         const __grid_constant__ CUtensorMap mapB, const Params p) {
@@ -724,6 +733,54 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t a = acc_iter & 1u;
       if (!warp_wait(&sh.tfull[a], (acc_iter >> 1) & 1u, sh, p, false, GG_EPI_BACKOFF_NS)) break;
       ptx::tc_fence_after();
+      float s_row = 1.f;  // per-row bias scale (read only for rows inside the group)
+      if (p.bias != nullptr && p.bias_scale != nullptr && row_ok) s_row = p.bias_scale[orow];
+      const __nv_bfloat16* bias_e =
+          p.bias != nullptr ? p.bias + (int64_t)tl.e * p.bias_ld : nullptr;
+      if constexpr (ACT == 1) {
+        // SiLU-and-mul: this warp owns output columns [oc, oc + CW/2) of the tile; their gate
+        // values are accumulator columns c_off/2 + j and their up values BN/2 further on
+        const int32_t half = c_off / 2;
+        const uint32_t tg = tmem_base + ((q * 32u) << 16) + a * BN + (uint32_t)half;
+        const int32_t oc = tl.n0 / 2 + half;
+#pragma unroll 1
+        for (int c = 0; c < CW / 2; c += 32) {
+          uint32_t rg[32], ru[32];
+          ptx::tmem_ld_32x32b_x32(tg + c, rg);
+          ptx::tmem_ld_32x32b_x32(tg + BN / 2 + c, ru);
+          ptx::tmem_ld_wait();
+          const int32_t col = oc + c;  // output column of rg[0]
+          if (row_ok && col < p.out_cols) {
+            uint32_t packed[16];
+#pragma unroll
+            for (int h = 0; h < 16; ++h) {
+              float v2[2];
+#pragma unroll
+              for (int u = 0; u < 2; ++u) {
+                const int i = 2 * h + u;
+                float g = __uint_as_float(rg[i]), up = __uint_as_float(ru[i]);
+                if (bias_e != nullptr) {
+                  g = fmaf(s_row, __bfloat162float(bias_e[tl.n0 + half + c + i]), g);
+                  up = fmaf(s_row, __bfloat162float(bias_e[tl.n0 + BN / 2 + half + c + i]), up);
+                }
+                v2[u] = g / (1.f + __expf(-g)) * up;
+              }
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(v2[0], v2[1]);
+              packed[h] = *reinterpret_cast<uint32_t*>(&b2);
+            }
+            __nv_bfloat16* dst = orow_ptr + col;
+            if (v8) {
+              ptx::st_global_v8(dst, packed);
+              ptx::st_global_v8(dst + 16, packed + 8);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                *reinterpret_cast<uint4*>(dst + 8 * j) = make_uint4(
+                    packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+            }
+          }
+        }
+      } else {
       const uint32_t taddr = tmem_base + ((q * 32u) << 16) + a * BN + (uint32_t)c_off;
       // 32 columns per load; the next load is in flight while this chunk is stored
       uint32_t r0[32], r1[32];
@@ -756,6 +813,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
         } else if (row_ok) {
+          if (bias_e != nullptr && col0 + c < p.out_cols) {
+            // h = product + s_row * bias[e, col]; out_cols is a multiple of 8, so a 32-wide
+            // chunk is read only up to its last valid 8-column group
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              if (col0 + c + 8 * j < p.out_cols) {
+                const uint4 bv = *reinterpret_cast<const uint4*>(bias_e + col0 + c + 8 * j);
+                const __nv_bfloat16* bb = reinterpret_cast<const __nv_bfloat16*>(&bv);
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                  cur[8 * j + u] = __float_as_uint(
+                      fmaf(s_row, __bfloat162float(bb[u]), __uint_as_float(cur[8 * j + u])));
+              }
+            }
+          }
           uint32_t packed[16];
 #pragma unroll
           for (int h = 0; h < 16; ++h) {
@@ -780,6 +852,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
+      }  // ACT
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) {

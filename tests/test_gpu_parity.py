@@ -223,3 +223,49 @@ def test_wgrad_f32_accumulates_over_two_calls():
     ref = 2.0 * oracle.wgrad(oracle.as_u16(r.A), oracle.as_u16(r.dY), r.offs, ks=ks)
     got = dW[:, torch.from_numpy(ks).cuda(), :].double().cpu().numpy()
     assert_close(got, ref, "wgrad_f32 accumulated twice")
+
+
+@pytest.mark.parametrize("act,with_bias,with_scale", [(0, True, False), (0, True, True),
+                                                      (1, False, False), (1, True, True)])
+def test_forward_epilogue_bias_scale_silu(act, with_bias, with_scale, variant):
+    """Fused epilogue: h = A W[e] + s[r] bias[e]; SiLU-and-mul over gate/up blocks of 128.
+    Rows past the last offset keep their sentinel and their NaN scale entries are not read."""
+    sizes = [0, 1, 127, 128, 129, 300, 17]
+    K, N = 192, 512
+    r = workloads.make_ragged_custom(len(sizes), K, N, sizes, seed=81, tail=40)
+    A, W = r.A.cuda(), r.W.cuda()
+    offs = torch.from_numpy(r.offs).cuda()
+    g = torch.Generator().manual_seed(5)
+    bias = torch.randn(r.E, N, generator=g).to(torch.bfloat16) if with_bias else None
+    scale = None
+    if with_scale:
+        scale = torch.randn(r.rows_alloc, generator=g, dtype=torch.float32)
+        scale[r.T:] = float("nan")  # capacity rows: never read
+    ncols = N // 2 if act == 1 else N
+    out = sentinel((r.rows_alloc, ncols))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    gg.forward_ex(A, W, offs, out, bias=None if bias is None else bias.cuda(),
+                  bias_scale=None if scale is None else scale.cuda(), act=act, status=st)
+    torch.cuda.synchronize()
+    s = int(st.item())
+    assert s & gg.DEV_LAUNCHED and (s & gg.DEV_ERROR_MASK) == 0
+    ref, grp = oracle.forward_ex(r.A, r.W, r.offs, bias,
+                                 None if scale is None else scale.numpy(), act)
+    T = r.T
+    assert_close(to_f64(out[:T]), ref[:T], "forward_ex")
+    assert bool(is_sentinel(out[T:]).all())
+
+
+def test_masked_forward_silu_mul_on_the_sglang_shape():
+    """The masked down-GEMM input: gate-up GEMM of the masked layout with fused SiLU-and-mul,
+    written only for the active rows (inactive rows NaN in A, sentinel in out)."""
+    m = workloads.make_masked(E=8, mmax=128, K=768, N=1536, seed=83)
+    bias = torch.randn(8, 1536).to(torch.bfloat16)
+    out = sentinel((8, 128, 768))
+    gg.masked_forward_ex(m.A.cuda(), m.W.cuda(), torch.from_numpy(m.masked_m).cuda(), out,
+                         bias=bias.cuda(), act=gg.ACT_SILU_MUL)
+    torch.cuda.synchronize()
+    ref, act, _ = oracle.masked_forward_ex(m.A, m.W, m.masked_m, bias, None, 1)
+    flat = out.view(-1, 768)
+    assert_close(to_f64(flat[torch.from_numpy(np.nonzero(act)[0]).cuda()]), ref[act], "masked silu")
+    assert bool(is_sentinel(flat[torch.from_numpy(np.nonzero(~act)[0]).cuda()]).all())

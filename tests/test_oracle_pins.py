@@ -330,3 +330,40 @@ def test_wgrad_accumulate_reduces_and_is_exact_on_integers():
     got = oracle.wgrad_accumulate(A, dY, offs, np.full((3, 4, 8), 3.0, np.float32), 0.5, -1.0)
     for e, m in enumerate([5, 0, 9]):
         assert np.all(got[e] == 0.5 * 2 * m - 3.0)
+
+
+def test_epilogue_bias_and_scale_reduce_exactly():
+    """Zero weights leave s[r]*bias[e] exactly; no bias and act 0 is the plain forward."""
+    sizes = [3, 0, 5]
+    r = workloads.make_ragged_custom(3, 16, 256, sizes, seed=77, tail=2)
+    bias = torch.randn(3, 256).to(torch.bfloat16)
+    scale = np.linspace(-2, 2, r.rows_alloc)
+    out, g = oracle.forward_ex(r.A, torch.zeros_like(r.W), r.offs, bias, scale)
+    b = _f64(bias)
+    for row in range(r.T):
+        assert np.all(out[row] == scale[row] * b[g[row]])
+    plain, _ = oracle.forward(r.A, r.W, r.offs)
+    same, _ = oracle.forward_ex(r.A, r.W, r.offs)
+    np.testing.assert_array_equal(same, plain)
+
+
+def test_epilogue_silu_mul_layout_and_closed_form():
+    """A one-hot, W[0,0,n] a distinct bf16-exact label per column: output column 128b+i must
+    be silu(gate) * up of gate column 256b+i and up column 256b+128+i (silu by math.exp)."""
+    import math
+    N, K = 512, 16
+    A = torch.zeros(4, K, dtype=torch.bfloat16)
+    A[:, 0] = 1
+    n = torch.arange(N, dtype=torch.float32)
+    labels = torch.where(n < 256, n / 64.0, (n - 384.0) / 64.0)  # <= 8 significant bits
+    W = torch.zeros(1, K, N, dtype=torch.bfloat16)
+    W[0, 0, :] = labels
+    assert torch.equal(W[0, 0].float(), labels)
+    out, _ = oracle.forward_ex(A, W, [4], act=1)
+    assert out.shape == (4, N // 2)
+    for b in range(N // 256):
+        for i in range(128):
+            gte = float(labels[256 * b + i])
+            up = float(labels[256 * b + 128 + i])
+            want = gte / (1.0 + math.exp(-gte)) * up
+            assert abs(out[3, 128 * b + i] - want) <= 1e-15 * max(1.0, abs(want))
