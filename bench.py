@@ -289,6 +289,10 @@ def run_ours(args):
     ms_per_step = total_ms / args.steps
     value = ws * step_flops / (ms_per_step * 1e-3) / 1e12
 
+    extras = None
+    if not args.no_extras:
+        extras = run_extras(args, gg, r, dev, stream, offs, out, dW)
+
     # end to end through the public API: pinned host inputs -> device, all passes, results
     # back to pinned host memory, every step inside the timed region
     e2e = None
@@ -337,6 +341,7 @@ def run_ours(args):
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,
+            "extras": extras,
             "gpu_launches": 4 * args.steps,
             "clocks": clocks,
         }
@@ -344,6 +349,61 @@ def run_ours(args):
     if ws > 1:
         torch.distributed.destroy_process_group()
     return 0
+
+
+def run_extras(args, gg, r, dev, stream, offs, out, dW):
+    """The further operations of the library on the same workload, each timed on its own
+    (outside the step): fp32 wgrad accumulating into a main-grad buffer (beta=1), forward
+    with per-expert bias and per-token bias scale, and forward with SiLU-and-mul."""
+    reps = max(3, args.steps // 2)
+    gen = torch.Generator(device=dev).manual_seed(11)
+    bias = torch.randn(r.E, r.N, generator=gen, device=dev).to(torch.bfloat16)
+    scale = torch.rand(r.rows_alloc, generator=gen, device=dev)
+    dw32 = torch.zeros((r.E, r.K, r.N), dtype=torch.float32, device=dev)
+    ops = {
+        "wgrad_f32_accumulate": lambda: gg.wgrad_f32(r.A, r.dY, offs, dw32, alpha=1.0, beta=1.0),
+        "forward_bias_scale": lambda: gg.forward_ex(r.A, r.W, offs, out, bias=bias,
+                                                    bias_scale=scale),
+    }
+    if r.N % 256 == 0:
+        act_out = torch.empty((r.rows_alloc, r.N // 2), dtype=torch.bfloat16, device=dev)
+        ops["forward_silu_mul"] = lambda: gg.forward_ex(r.A, r.W, offs, act_out, bias=bias,
+                                                        act=gg.ACT_SILU_MUL)
+    # token routing that would produce this workload's packed rows: T/8 tokens, top-8
+    tok = max(1, r.T // 8)
+    ids_np, X = __import__("workloads").make_routing(tok, 8, r.E, r.K, seed=12, device=dev) \
+        if tok <= 65536 else (None, None)
+    route_bytes = None
+    if ids_np is not None:
+        ids = torch.from_numpy(ids_np).to(dev)
+        a_packed = torch.empty((tok * 8, r.K), dtype=torch.bfloat16, device=dev)
+        row_of = torch.empty(tok * 8, dtype=torch.int32, device=dev)
+        roffs = torch.empty(r.E, dtype=torch.int32, device=dev)
+        ws = torch.empty(max(4, gg.route_workspace_bytes(tok * 8, r.E)), dtype=torch.uint8,
+                         device=dev)
+        ops["route_tokens"] = lambda: gg.route(ids, X, r.E, A_packed=a_packed, row_of=row_of,
+                                               offs=roffs, workspace=ws)
+        # ids + X once + packed rows + row_of + offsets
+        route_bytes = (ids.numel() * 4 + X.numel() * 2 + a_packed.numel() * 2
+                       + row_of.numel() * 4 + r.E * 4)
+    res = {}
+    for name, fn in ops.items():
+        fn()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        if name == "route_tokens":
+            res[name] = {"ms": ms, "gbs": route_bytes / (ms * 1e-3) / 1e9,
+                         "tokens": tok, "topk": 8, "launches": 3 * reps}
+        else:
+            res[name] = {"ms": ms, "tflops": r.flops / (ms * 1e-3) / 1e12, "launches": reps}
+    return res
 
 
 def run_e2e(args, gg, r, m, dev, stream, ws, barrier):
@@ -411,6 +471,7 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--variant", type=int, default=0, choices=[0, 1, 2],
                     help="launch shape of forward/dgrad: 0 automatic, 1 single CTA, 2 CTA pair")
     args = ap.parse_args(argv)

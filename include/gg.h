@@ -44,6 +44,7 @@
 #ifndef GG_H_
 #define GG_H_
 
+#include <stddef.h>
 #include <stdint.h>
 #include <cuda_runtime.h>
 
@@ -72,6 +73,8 @@ typedef enum {
 #define GG_DEV_BAD_MASKED_M 0x2u  /* a masked_m was < 0 or > mmax; it was clamped         */
 #define GG_DEV_TIMEOUT      0x4u  /* a pipeline wait exceeded the watchdog; results of this
                                      call are incomplete                                  */
+#define GG_DEV_BAD_ROUTE    0x8u  /* gg_route: an expert id was >= E; that assignment was
+                                     dropped                                              */
 #define GG_DEV_ERROR_MASK   0xFFu
 #define GG_DEV_LAUNCHED     0x100u /* informational: the sm_100a kernel ran to its end     */
 
@@ -173,6 +176,26 @@ GG_API gg_status gg_masked_forward_ex(const void* A, const void* W, const int32_
                                       void* out, int64_t mmax, int64_t K, int64_t N, int32_t E,
                                       const gg_epilogue* epi, int32_t* dev_status,
                                       cudaStream_t stream);
+
+/*
+ * Token routing into the packed layout of the grouped GEMM (the step before the path: it
+ * plays the part of torchtitan's generate_permute_indices in PyTorch issue 152668, without
+ * the alignment padding that issue relies on, and without a host round trip).
+ *   topk_ids int32 [T_tok, k], device: expert of assignment i = t*k + s; ids < 0 mean
+ *            "dropped", ids >= E are dropped and flag GG_DEV_BAD_ROUTE
+ *   X        bf16 [T_tok, K]; A_packed bf16 [T_tok*k, K] (only its first offs[E-1] rows are
+ *            written: row_of[i] of assignment i gets a copy of X[t])
+ *   row_of   int32 [T_tok*k]: packed row of each assignment, -1 when dropped
+ *   offs     int32 [E]: cumulative end offsets, ready for gg_forward & co.
+ * Rows are ordered by expert and, inside an expert, by assignment index (a stable sort), so
+ * the result is deterministic. `workspace` is caller-owned device memory of at least
+ * gg_route_workspace_bytes(T_tok*k, E) bytes (4-byte aligned); it need not be cleared.
+ */
+GG_API size_t gg_route_workspace_bytes(int64_t n_assign, int32_t E);
+GG_API gg_status gg_route(const int32_t* topk_ids, int64_t T_tok, int32_t k, int32_t E,
+                          const void* X, int64_t K, void* A_packed, int32_t* row_of,
+                          int32_t* offs, void* workspace, size_t workspace_bytes,
+                          int32_t* dev_status, cudaStream_t stream);
 
 /* A static, human-readable name for a status. */
 GG_API const char* gg_status_string(gg_status s);

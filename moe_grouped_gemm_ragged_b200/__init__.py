@@ -25,6 +25,7 @@ GG_OK, GG_ERR_INVALID_ARG, GG_ERR_UNSUPPORTED, GG_ERR_CUDA = 0, 1, 2, 3
 DEV_BAD_OFFSETS = 0x1
 DEV_BAD_MASKED_M = 0x2
 DEV_TIMEOUT = 0x4
+DEV_BAD_ROUTE = 0x8
 DEV_ERROR_MASK = 0xFF
 DEV_LAUNCHED = 0x100
 MAX_EXPERTS = 1024
@@ -71,6 +72,10 @@ def lib() -> ctypes.CDLL:
     L.gg_masked_forward_ex.argtypes = [P, P, P, P, i64, i64, i64, i32,
                                        ctypes.POINTER(_Epilogue), P, P]
     L.gg_masked_forward_ex.restype = ctypes.c_int
+    L.gg_route_workspace_bytes.argtypes = [i64, i32]
+    L.gg_route_workspace_bytes.restype = ctypes.c_size_t
+    L.gg_route.argtypes = [P, i64, i32, i32, P, i64, P, P, P, P, ctypes.c_size_t, P, P]
+    L.gg_route.restype = ctypes.c_int
     L.gg_status_string.argtypes = [ctypes.c_int]
     L.gg_status_string.restype = ctypes.c_char_p
     L.gg_set_watchdog_ns.argtypes = [ctypes.c_uint64]
@@ -302,6 +307,42 @@ def masked_forward(A: torch.Tensor, W: torch.Tensor, masked_m: torch.Tensor,
     return out
 
 
+def route_workspace_bytes(n_assign: int, E: int) -> int:
+    return int(lib().gg_route_workspace_bytes(int(n_assign), int(E)))
+
+
+def route(topk_ids: torch.Tensor, X: torch.Tensor, E: int, *,
+          A_packed: Optional[torch.Tensor] = None, row_of: Optional[torch.Tensor] = None,
+          offs: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+          status: Optional[torch.Tensor] = None, stream=None):
+    """Token routing into the packed grouped-GEMM layout. Returns (A_packed [T*k, K],
+    row_of [T*k], offs [E]); buffers left as None are allocated (uninitialised)."""
+    _check(topk_ids, "topk_ids", torch.int32, 2)
+    _check(X, "X", torch.bfloat16, 2)
+    T, k = topk_ids.shape
+    T2, K = X.shape
+    if T2 != T:
+        raise ValueError("topk_ids[T, k] and X[T, K] disagree on T")
+    n = T * k
+    dev = X.device
+    A_packed = torch.empty((n, K), dtype=X.dtype, device=dev) if A_packed is None else A_packed
+    row_of = torch.empty(n, dtype=torch.int32, device=dev) if row_of is None else row_of
+    offs = torch.empty(E, dtype=torch.int32, device=dev) if offs is None else offs
+    wb = route_workspace_bytes(n, E)
+    if workspace is None:
+        workspace = torch.empty(max(wb, 4), dtype=torch.uint8, device=dev)
+    _check(A_packed, "A_packed", torch.bfloat16, 2)
+    _check(row_of, "row_of", torch.int32, 1)
+    _check(offs, "offs", torch.int32, 1)
+    if tuple(A_packed.shape) != (n, K) or row_of.numel() != n or offs.numel() != E:
+        raise ValueError("shape mismatch: A_packed[T*k, K], row_of[T*k], offs[E]")
+    rc = lib().gg_route(_ptr(topk_ids), T, k, E, _ptr(X), K, _ptr(A_packed), _ptr(row_of),
+                        _ptr(offs), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                        _status_ptr(status), _stream_handle(stream))
+    _raise(rc, "gg_route")
+    return A_packed, row_of, offs
+
+
 def grouped_mm(A: torch.Tensor, W: torch.Tensor, offs: torch.Tensor,
                out: Optional[torch.Tensor] = None, **kw) -> torch.Tensor:
     """Forward with an optional caller-owned ``out`` (allocated uninitialised when None)."""
@@ -312,7 +353,7 @@ def grouped_mm(A: torch.Tensor, W: torch.Tensor, offs: torch.Tensor,
 
 __all__ = [
     "forward", "forward_ex", "dgrad", "wgrad", "wgrad_f32", "masked_forward",
-    "masked_forward_ex", "ACT_NONE", "ACT_SILU_MUL", "grouped_mm", "status_string", "version",
+    "masked_forward_ex", "ACT_NONE", "ACT_SILU_MUL", "route", "route_workspace_bytes", "grouped_mm", "status_string", "version",
     "set_watchdog_ns", "testing_skip_first_load", "testing_force_variant", "lib", "GGError", "LIB_PATH",
     "DEV_BAD_OFFSETS", "DEV_BAD_MASKED_M", "DEV_TIMEOUT", "DEV_ERROR_MASK", "DEV_LAUNCHED",
     "MAX_EXPERTS",

@@ -1,0 +1,176 @@
+// Token routing into the packed layout of the ragged grouped GEMM: per-expert cumulative end
+// offsets, the packed row of every (token, slot) assignment and the packed activations,
+// all on the device. A stable counting sort over the flattened assignments in three
+// launches: per-block histograms, one scan, and a scatter that also copies the rows.
+#include <cstdint>
+#include <cstring>
+
+#include <cuda_runtime.h>
+
+#include "gg.h"
+
+namespace ggr {
+
+constexpr int THREADS = 256;          // one assignment per thread and block
+constexpr int WARPS = THREADS / 32;
+constexpr int CHUNK = THREADS;        // assignments per block
+constexpr int32_t DEV_BAD_ROUTE = 0x8;
+static_assert(DEV_BAD_ROUTE == GG_DEV_BAD_ROUTE, "status bit mismatch");
+
+// Histogram of the block's chunk: counts[b * E + e] (ids < 0 are dropped silently, ids >= E
+// are dropped and flagged).
+__global__ void __launch_bounds__(THREADS) count_kernel(const int32_t* __restrict__ ids,
+                                                        int64_t n, int32_t E,
+                                                        int32_t* __restrict__ counts,
+                                                        int32_t* status) {
+  __shared__ int32_t hist[GG_MAX_EXPERTS];
+  for (int e = threadIdx.x; e < E; e += THREADS) hist[e] = 0;
+  __syncthreads();
+  const int64_t i = (int64_t)blockIdx.x * CHUNK + threadIdx.x;
+  bool bad = false;
+  if (i < n) {
+    const int32_t e = ids[i];
+    if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
+    bad = e >= E;
+  }
+  bad = __syncthreads_or(bad);
+  for (int e = threadIdx.x; e < E; e += THREADS) counts[(int64_t)blockIdx.x * E + e] = hist[e];
+  if (bad && threadIdx.x == 0 && status != nullptr) atomicOr(status, DEV_BAD_ROUTE);
+}
+
+// One block: offs[e] = cumulative end of expert e; counts[b][e] becomes the first packed row
+// of block b's assignments to expert e.
+__global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ counts, int32_t nblk,
+                                                    int32_t E, int32_t* __restrict__ offs) {
+  __shared__ int32_t warp_sum[32];
+  const int e = threadIdx.x;
+  int32_t total = 0;
+  if (e < E)
+    for (int32_t b = 0; b < nblk; ++b) total += counts[(int64_t)b * E + e];
+  // block-wide inclusive scan of total over e
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int32_t v = total;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int32_t o = __shfl_up_sync(0xffffffffu, v, d);
+    if (lane >= d) v += o;
+  }
+  if (lane == 31) warp_sum[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    int32_t w = warp_sum[lane];
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int32_t o = __shfl_up_sync(0xffffffffu, w, d);
+      if (lane >= d) w += o;
+    }
+    warp_sum[lane] = w;
+  }
+  __syncthreads();
+  const int32_t incl = v + (warp > 0 ? warp_sum[warp - 1] : 0);
+  if (e < E) {
+    offs[e] = incl;
+    int32_t run = incl - total;
+    for (int32_t b = 0; b < nblk; ++b) {
+      const int32_t c = counts[(int64_t)b * E + e];
+      counts[(int64_t)b * E + e] = run;
+      run += c;
+    }
+  }
+}
+
+// Stable ranks inside the block (warp by warp, lane by lane), row_of, and the row copies.
+__global__ void __launch_bounds__(THREADS) scatter_kernel(
+    const int32_t* __restrict__ ids, int64_t n, int32_t k, int32_t E,
+    const int32_t* __restrict__ bases, const uint4* __restrict__ X, int64_t row_vecs,
+    uint4* __restrict__ A_packed, int32_t* __restrict__ row_of) {
+  extern __shared__ int32_t whist[];  // [WARPS][E]: per-warp counts, then per-warp bases
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < WARPS * E; i += THREADS) whist[i] = 0;
+  __syncthreads();
+  const int64_t i = (int64_t)blockIdx.x * CHUNK + threadIdx.x;
+  const int32_t e = i < n ? ids[i] : -1;
+  const bool valid = e >= 0 && e < E;
+  // lanes with the same expert form one peer set; an invalid lane is alone
+  const uint32_t peers = __match_any_sync(0xffffffffu, valid ? e : -1 - lane);
+  const uint32_t rank = __popc(peers & ((1u << lane) - 1u));
+  if (valid && rank == 0) whist[warp * E + e] = __popc(peers);
+  __syncthreads();
+  // exclusive scan over warps per expert, starting at the block's base
+  for (int x = threadIdx.x; x < E; x += THREADS) {
+    int32_t run = bases[(int64_t)blockIdx.x * E + x];
+    for (int w = 0; w < WARPS; ++w) {
+      const int32_t c = whist[w * E + x];
+      whist[w * E + x] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  const int32_t dest = valid ? whist[warp * E + e] + (int32_t)rank : -1;
+  if (i < n) row_of[i] = dest;
+  // the warp copies its 32 rows, one after the other, each with all lanes
+  const int64_t tok = i / k;
+  for (int j = 0; j < 32; ++j) {
+    const int32_t d = __shfl_sync(0xffffffffu, dest, j);
+    const int64_t t = __shfl_sync(0xffffffffu, tok, j);
+    if (d < 0) continue;
+    const uint4* src = X + t * row_vecs;
+    uint4* dst = A_packed + (int64_t)d * row_vecs;
+    for (int64_t v = lane; v < row_vecs; v += 32) dst[v] = src[v];
+  }
+}
+
+int64_t blocks_for(int64_t n) { return (n + CHUNK - 1) / CHUNK; }
+
+}  // namespace ggr
+
+extern "C" {
+
+size_t gg_route_workspace_bytes(int64_t n_assign, int32_t E) {
+  if (n_assign < 0 || E < 1) return 0;
+  return (size_t)ggr::blocks_for(n_assign) * (size_t)E * sizeof(int32_t);
+}
+
+gg_status gg_route(const int32_t* topk_ids, int64_t T_tok, int32_t k, int32_t E, const void* X,
+                   int64_t K, void* A_packed, int32_t* row_of, int32_t* offs, void* workspace,
+                   size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream) {
+  using namespace ggr;
+  if (T_tok < 0 || k < 1 || E < 1 || K < 1) return GG_ERR_INVALID_ARG;
+  if (E > GG_MAX_EXPERTS) return GG_ERR_UNSUPPORTED;
+  if (K % 8 != 0) return GG_ERR_UNSUPPORTED;
+  const int64_t n = T_tok * (int64_t)k;
+  if (n >= (int64_t(1) << 31)) return GG_ERR_UNSUPPORTED;
+  if (offs == nullptr) return GG_ERR_INVALID_ARG;
+  if (n > 0 && (topk_ids == nullptr || X == nullptr || A_packed == nullptr ||
+                row_of == nullptr || workspace == nullptr))
+    return GG_ERR_INVALID_ARG;
+  auto mis = [](const void* p, uintptr_t a) {
+    return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0;
+  };
+  if (mis(topk_ids, 4) || mis(row_of, 4) || mis(offs, 4) || mis(workspace, 4) ||
+      mis(X, 16) || mis(A_packed, 16) || (dev_status != nullptr && mis(dev_status, 4)))
+    return GG_ERR_UNSUPPORTED;
+  if (workspace_bytes < gg_route_workspace_bytes(n, E)) return GG_ERR_INVALID_ARG;
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return GG_ERR_CUDA;
+  if (major != 10) return GG_ERR_UNSUPPORTED;
+  const int64_t nblk = blocks_for(n);
+  int32_t* counts = reinterpret_cast<int32_t*>(workspace);
+  if (nblk > 0)
+    count_kernel<<<(unsigned)nblk, THREADS, 0, stream>>>(topk_ids, n, E, counts, dev_status);
+  scan_kernel<<<1, 1024, 0, stream>>>(counts, (int32_t)nblk, E, offs);  // nblk 0: offs = 0
+  if (nblk == 0) return cudaGetLastError() == cudaSuccess ? GG_OK : GG_ERR_CUDA;
+  const size_t smem = sizeof(int32_t) * WARPS * (size_t)E;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return GG_ERR_CUDA;
+  scatter_kernel<<<(unsigned)nblk, THREADS, smem, stream>>>(
+      topk_ids, n, k, E, counts, reinterpret_cast<const uint4*>(X), K / 8,
+      reinterpret_cast<uint4*>(A_packed), row_of);
+  return cudaGetLastError() == cudaSuccess ? GG_OK : GG_ERR_CUDA;
+}
+
+}  // extern "C"

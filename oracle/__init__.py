@@ -217,6 +217,26 @@ def masked_forward_ex(A, W, masked_m, bias=None, bias_scale=None, act: int = 0, 
     return epilogue(h, g, r, bias, bias_scale, act), act_rows, bad
 
 
+def route(topk_ids, X, E: int):
+    """Token routing into the packed grouped-GEMM layout (the step before the path:
+    torchtitan's generate_permute_indices in PyTorch issue 152668, here without alignment
+    padding). Assignment i = t*k + s sends token t to expert topk_ids[t, s]; ids < 0 or
+    >= E are dropped. Rows are ordered by expert, and within an expert by assignment index
+    (a stable sort). Returns (offs int32[E] cumulative ends, row_of int32[T*k] with -1 for
+    dropped assignments, A_packed bf16-as-uint16 [total, K], bad: any id >= E)."""
+    ids = np.asarray(topk_ids, dtype=np.int64).reshape(-1)
+    Xu = as_u16(X)
+    k = np.asarray(topk_ids).shape[1]
+    valid = (ids >= 0) & (ids < E)
+    order = np.argsort(np.where(valid, ids, E), kind="stable")[: int(valid.sum())]
+    counts = np.bincount(ids[valid], minlength=E)
+    offs = np.cumsum(counts).astype(np.int32)
+    row_of = np.full(len(ids), -1, np.int32)
+    row_of[order] = np.arange(len(order), dtype=np.int32)
+    A_packed = Xu[order // k]
+    return offs, row_of, A_packed, bool(np.any(ids >= E))
+
+
 def masked_forward(A, W, masked_m, rows=None, threads=None):
     """fp64 masked forward on flat rows e*mmax+r (default: all). Returns
     (out[nrows,N], active[nrows], bad)."""

@@ -367,3 +367,38 @@ def test_epilogue_silu_mul_layout_and_closed_form():
             up = float(labels[256 * b + 128 + i])
             want = gte / (1.0 + math.exp(-gte)) * up
             assert abs(out[3, 128 * b + i] - want) <= 1e-15 * max(1.0, abs(want))
+
+
+def _route_brute(ids, X, E):
+    """Obviously-correct routing: for each expert in order, every assignment in order."""
+    ids = np.asarray(ids)
+    T, k = ids.shape
+    rows, row_of, offs = [], np.full(T * k, -1, np.int32), []
+    for e in range(E):
+        for t in range(T):
+            for s in range(k):
+                if ids[t, s] == e:
+                    row_of[t * k + s] = len(rows)
+                    rows.append(t)
+        offs.append(len(rows))
+    Xu = oracle.as_u16(X)
+    return np.array(offs, np.int32), row_of, Xu[rows] if rows else Xu[:0]
+
+
+def test_route_matches_brute_force_and_invariants():
+    ids, X = workloads.make_routing(37, 3, 6, 16, seed=5, dropped=4)
+    ids[0, 0] = 9  # out of range: dropped and flagged
+    offs, row_of, Ap, bad = oracle.route(ids, X, 6)
+    boffs, brow, bA = _route_brute(ids, X, 6)
+    np.testing.assert_array_equal(offs, boffs)
+    np.testing.assert_array_equal(row_of, brow)
+    np.testing.assert_array_equal(Ap, bA)
+    assert bad
+    # every packed row of group e came from an assignment to expert e
+    flat = ids.reshape(-1)
+    starts = np.concatenate([[0], offs[:-1]])
+    for i, r in enumerate(row_of):
+        if r >= 0:
+            e = flat[i]
+            assert starts[e] <= r < offs[e]
+    assert offs[-1] == np.count_nonzero((flat >= 0) & (flat < 6))

@@ -240,3 +240,21 @@ def make_masked(*, seed: int = 2, nan_inactive: bool = True, device="cpu",
             lo = int(min(max(int(m[e]), 0), mmax))
             A[e, lo:] = float("nan")
     return MaskedInputs(E, mmax, K, N, m, A, W)
+
+
+def make_routing(T_tok: int, k: int, E: int, K: int, *, seed: int, zipf: float = 1.2,
+                 dropped: int = 0, device="cpu"):
+    """Top-k routing of T_tok tokens over E experts: each token picks k distinct experts with
+    Zipf(zipf) popularity over a seeded random rank order; `dropped` assignments get id -1.
+    Returns (topk_ids int32 [T_tok, k], X bf16 [T_tok, K])."""
+    rng = np.random.default_rng(seed)
+    ranks = rng.permutation(E) + 1
+    p = ranks.astype(np.float64) ** -zipf
+    p /= p.sum()
+    ids = np.stack([rng.choice(E, k, replace=False, p=p) for _ in range(T_tok)]).astype(np.int32)
+    if dropped:
+        flat = ids.reshape(-1)
+        flat[rng.choice(flat.size, dropped, replace=False)] = -1
+    gen = torch.Generator(device=device).manual_seed(seed)
+    X = _randn_bf16((T_tok, K), gen, device)
+    return ids, X
