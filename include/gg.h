@@ -63,7 +63,9 @@ typedef enum {
   GG_ERR_INVALID_ARG = 1,  /* null pointer, negative or zero size, E < 1, ...          */
   GG_ERR_UNSUPPORTED = 2,  /* K or N not a multiple of 8, misaligned pointer, E too large,
                               rows >= 2^31, or a device that is not sm_100                */
-  GG_ERR_CUDA = 3          /* a CUDA runtime/driver call failed (launch, attribute, ...) */
+  GG_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed (launch, attribute, ...) */
+  GG_ERR_TOO_LARGE = 4     /* gg_route_noalloc: the problem needs more than its fixed
+                              scratch array (GG_ROUTE_NOALLOC_MAX_COUNTS entries)          */
 } gg_status;
 
 /* Bits OR-ed into *dev_status by the kernels. */
@@ -196,6 +198,27 @@ GG_API gg_status gg_route(const int32_t* topk_ids, int64_t T_tok, int32_t k, int
                           const void* X, int64_t K, void* A_packed, int32_t* row_of,
                           int32_t* offs, void* workspace, size_t workspace_bytes,
                           int32_t* dev_status, cudaStream_t stream);
+
+/*
+ * gg_route without a workspace argument, for callers that cannot allocate device memory
+ * where they route tokens (for example a runtime whose device memory is reserved up front
+ * by its own allocator, or code that must not enter the CUDA allocator at that point). The
+ * pages have no counterpart of this entry point.
+ * Same arguments, results and status bits as gg_route, minus the workspace. Instead of a
+ * workspace the per-block histograms use one fixed device array inside the library:
+ * GG_ROUTE_NOALLOC_MAX_COUNTS int32 entries (1 MiB), held by every GPU that loads the library
+ * until the process exits. A call needs ceil(T_tok*k / 256) * E entries; larger problems
+ * return GG_ERR_TOO_LARGE (e.g. at most 65536 assignments with 1024 experts, 1048576 with
+ * 64). Nothing is allocated, freed or cleared: every entry a call reads it wrote itself.
+ * All calls share the array, so calls that overlap on the GPU (other streams, other threads)
+ * race; order them on one stream. The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress) with that device current; make that first call before any
+ * stream capture.
+ */
+#define GG_ROUTE_NOALLOC_MAX_COUNTS (1 << 18)
+GG_API gg_status gg_route_noalloc(const int32_t* topk_ids, int64_t T_tok, int32_t k, int32_t E,
+                                  const void* X, int64_t K, void* A_packed, int32_t* row_of,
+                                  int32_t* offs, int32_t* dev_status, cudaStream_t stream);
 
 /* A static, human-readable name for a status. */
 GG_API const char* gg_status_string(gg_status s);

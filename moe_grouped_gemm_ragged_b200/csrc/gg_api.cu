@@ -465,6 +465,9 @@ const char* gg_status_string(gg_status s) {
     case GG_ERR_UNSUPPORTED:
       return "GG_ERR_UNSUPPORTED: unsupported device, alignment, size or expert count";
     case GG_ERR_CUDA: return "GG_ERR_CUDA: a CUDA runtime or driver call failed";
+    case GG_ERR_TOO_LARGE:
+      return "GG_ERR_TOO_LARGE: the problem needs more than the fixed scratch array of "
+             "gg_route_noalloc (GG_ROUTE_NOALLOC_MAX_COUNTS entries)";
   }
   return "unknown gg_status";
 }

@@ -4,6 +4,7 @@
 // launches: per-block histograms, one scan, and a scatter that also copies the rows.
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include <cuda_runtime.h>
 
@@ -161,6 +162,90 @@ gg_status gg_route(const int32_t* topk_ids, int64_t T_tok, int32_t k, int32_t E,
   if (nblk > 0)
     count_kernel<<<(unsigned)nblk, THREADS, 0, stream>>>(topk_ids, n, E, counts, dev_status);
   scan_kernel<<<1, 1024, 0, stream>>>(counts, (int32_t)nblk, E, offs);  // nblk 0: offs = 0
+  if (nblk == 0) return cudaGetLastError() == cudaSuccess ? GG_OK : GG_ERR_CUDA;
+  const size_t smem = sizeof(int32_t) * WARPS * (size_t)E;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return GG_ERR_CUDA;
+  scatter_kernel<<<(unsigned)nblk, THREADS, smem, stream>>>(
+      topk_ids, n, k, E, counts, reinterpret_cast<const uint4*>(X), K / 8,
+      reinterpret_cast<uint4*>(A_packed), row_of);
+  return cudaGetLastError() == cudaSuccess ? GG_OK : GG_ERR_CUDA;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- allocation-free routing
+// gg_route_noalloc serves callers that cannot allocate device memory where they call the
+// router (for example a runtime whose device memory is reserved up front by its own
+// allocator, or code that must not enter the CUDA allocator at that point). Its per-block
+// histograms live in this fixed array instead of a caller-provided workspace. Every GPU that
+// loads the library holds the array (1 MiB) until the process exits. Host code only sees a
+// stand-in for it, so its device address is looked up once per device with
+// cudaGetSymbolAddress while that device is current.
+static __device__ __align__(256) int32_t g_route_counts[GG_ROUTE_NOALLOC_MAX_COUNTS];
+
+namespace ggr {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+int32_t* g_noalloc_counts[kMaxDevices] = {};
+
+// Device address of g_route_counts on the current device (looked up on first use).
+gg_status noalloc_counts(int32_t** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GG_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return GG_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_counts[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_route_counts) != cudaSuccess || p == nullptr)
+      return GG_ERR_CUDA;
+    g_noalloc_counts[dev] = static_cast<int32_t*>(p);
+  }
+  *out = g_noalloc_counts[dev];
+  return GG_OK;
+}
+
+}  // namespace ggr
+
+extern "C" {
+
+gg_status gg_route_noalloc(const int32_t* topk_ids, int64_t T_tok, int32_t k, int32_t E,
+                           const void* X, int64_t K, void* A_packed, int32_t* row_of,
+                           int32_t* offs, int32_t* dev_status, cudaStream_t stream) {
+  using namespace ggr;
+  if (T_tok < 0 || k < 1 || E < 1 || K < 1) return GG_ERR_INVALID_ARG;
+  if (E > GG_MAX_EXPERTS) return GG_ERR_UNSUPPORTED;
+  if (K % 8 != 0) return GG_ERR_UNSUPPORTED;
+  const int64_t n = T_tok * (int64_t)k;
+  if (n >= (int64_t(1) << 31)) return GG_ERR_UNSUPPORTED;
+  const int64_t nblk = blocks_for(n);
+  if (nblk * (int64_t)E > GG_ROUTE_NOALLOC_MAX_COUNTS) return GG_ERR_TOO_LARGE;
+  if (offs == nullptr) return GG_ERR_INVALID_ARG;
+  if (n > 0 && (topk_ids == nullptr || X == nullptr || A_packed == nullptr ||
+                row_of == nullptr))
+    return GG_ERR_INVALID_ARG;
+  auto mis = [](const void* p, uintptr_t a) {
+    return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0;
+  };
+  if (mis(topk_ids, 4) || mis(row_of, 4) || mis(offs, 4) || mis(X, 16) || mis(A_packed, 16) ||
+      (dev_status != nullptr && mis(dev_status, 4)))
+    return GG_ERR_UNSUPPORTED;
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return GG_ERR_CUDA;
+  if (major != 10) return GG_ERR_UNSUPPORTED;
+  int32_t* counts = nullptr;
+  const gg_status s = noalloc_counts(&counts);
+  if (s != GG_OK) return s;
+  // The histogram kernel writes every entry the later kernels read, so the array needs no
+  // clearing; calls that overlap on the GPU share it and race.
+  if (nblk > 0)
+    count_kernel<<<(unsigned)nblk, THREADS, 0, stream>>>(topk_ids, n, E, counts, dev_status);
+  scan_kernel<<<1, 1024, 0, stream>>>(counts, (int32_t)nblk, E, offs);
   if (nblk == 0) return cudaGetLastError() == cudaSuccess ? GG_OK : GG_ERR_CUDA;
   const size_t smem = sizeof(int32_t) * WARPS * (size_t)E;
   if (smem > 48 * 1024 &&
