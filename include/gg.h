@@ -118,6 +118,17 @@ GG_API gg_status gg_wgrad(const void* A, const void* dY, const int32_t* offs, vo
                    int64_t rows_alloc, int64_t K, int64_t N, int32_t E,
                    int32_t* dev_status, cudaStream_t stream);
 
+/* gg_dgrad with flags: GG_FLAG_ZERO_TAIL (dX rows past the last offset become 0) and
+   GG_FLAG_W_NK (W is [E, N, K]). */
+GG_API gg_status gg_dgrad_ex(const void* dY, const void* W, const int32_t* offs, void* dX,
+                             int64_t rows_alloc, int64_t K, int64_t N, int32_t E,
+                             int32_t flags, int32_t* dev_status, cudaStream_t stream);
+
+/* gg_wgrad with flags: GG_FLAG_W_NK writes dW as [E, N, K] (dW[e] = dY_e^T . A_e). */
+GG_API gg_status gg_wgrad_ex(const void* A, const void* dY, const int32_t* offs, void* dW,
+                             int64_t rows_alloc, int64_t K, int64_t N, int32_t E,
+                             int32_t flags, int32_t* dev_status, cudaStream_t stream);
+
 /*
  * Wgrad into an fp32 buffer with scaling and accumulation (the main-grad update):
  *   dW[e, k, n] = alpha * sum over rows r of group e of A[r, k] * dY[r, n]
@@ -161,14 +172,25 @@ GG_API gg_status gg_masked_forward(const void* A, const void* W, const int32_t* 
  * (SiLU-and-mul between the gate-up and the down GEMM, written only for active rows). */
 #define GG_ACT_NONE 0
 #define GG_ACT_SILU_MUL 1
+/* Flags of the _ex entry points.
+ *   GG_FLAG_ZERO_TAIL  forward, dgrad: rows of out / dX at and past the last effective offset
+ *                      are written with zeros (a complete tensor, e.g. for autograd) instead
+ *                      of being left untouched
+ *   GG_FLAG_W_NK       W (and dW) stored [E, N, K]: each expert's weight out-major, the way
+ *                      TransformerEngine's GroupedLinear keeps it (TransformerEngine PR 3542,
+ *                      "Adds TN, NN, and NT dispatch"); forward computes A . W[e]^T */
+#define GG_FLAG_ZERO_TAIL 0x1
+#define GG_FLAG_W_NK 0x2
 typedef struct gg_epilogue {
   const void* bias;
   const float* bias_scale;
   int32_t act;
+  int32_t flags; /* GG_FLAG_ZERO_TAIL | GG_FLAG_W_NK */
 } gg_epilogue;
 
-/* gg_forward with a fused epilogue (epi may be NULL: same as gg_forward). out is
-   bf16 [rows_alloc, N] (GG_ACT_NONE) or [rows_alloc, N/2] (GG_ACT_SILU_MUL). */
+/* gg_forward with a fused epilogue and flags (epi may be NULL: same as gg_forward). out is
+   bf16 [rows_alloc, N] (GG_ACT_NONE) or [rows_alloc, N/2] (GG_ACT_SILU_MUL). With
+   GG_FLAG_W_NK, W is [E, N, K]. */
 GG_API gg_status gg_forward_ex(const void* A, const void* W, const int32_t* offs, void* out,
                                int64_t rows_alloc, int64_t K, int64_t N, int32_t E,
                                const gg_epilogue* epi, int32_t* dev_status, cudaStream_t stream);
@@ -237,6 +259,10 @@ GG_API int gg_testing_skip_first_load(int enable);
    2 = CTA pairs (256-row tiles on two SMs). Results are the same up to rounding order.
    Returns the previous setting. */
 GG_API int gg_testing_force_variant(int variant);
+
+/* Text of the CUDA failure behind the last GG_ERR_CUDA returned in this thread ("" if none).
+   The pointer stays valid until the thread's next call into the library. */
+GG_API const char* gg_last_error(void);
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 GG_API int gg_version(void);

@@ -33,11 +33,12 @@ MAX_EXPERTS = 1024
 _lib = None
 
 ACT_NONE, ACT_SILU_MUL = 0, 1
+FLAG_ZERO_TAIL, FLAG_W_NK = 0x1, 0x2
 
 
 class _Epilogue(ctypes.Structure):
     _fields_ = [("bias", ctypes.c_void_p), ("bias_scale", ctypes.c_void_p),
-                ("act", ctypes.c_int32)]
+                ("act", ctypes.c_int32), ("flags", ctypes.c_int32)]
 
 
 class GGError(RuntimeError):
@@ -45,7 +46,10 @@ class GGError(RuntimeError):
 
     def __init__(self, code: int, where: str):
         self.code = code
-        super().__init__(f"{where}: {status_string(code)}")
+        detail = ""
+        if code == GG_ERR_CUDA:
+            detail = " (" + lib().gg_last_error().decode() + ")"
+        super().__init__(f"{where}: {status_string(code)}{detail}")
 
 
 def lib() -> ctypes.CDLL:
@@ -67,6 +71,10 @@ def lib() -> ctypes.CDLL:
     L.gg_wgrad_f32.argtypes = [P, P, P, P, ctypes.c_float, ctypes.c_float, i64, i64, i64, i32,
                                P, P]
     L.gg_wgrad_f32.restype = ctypes.c_int
+    for name in ("gg_dgrad_ex", "gg_wgrad_ex"):
+        fn = getattr(L, name)
+        fn.argtypes = [P, P, P, P, i64, i64, i64, i32, i32, P, P]
+        fn.restype = ctypes.c_int
     L.gg_forward_ex.argtypes = [P, P, P, P, i64, i64, i64, i32, ctypes.POINTER(_Epilogue), P, P]
     L.gg_forward_ex.restype = ctypes.c_int
     L.gg_masked_forward_ex.argtypes = [P, P, P, P, i64, i64, i64, i32,
@@ -85,6 +93,7 @@ def lib() -> ctypes.CDLL:
     L.gg_testing_force_variant.argtypes = [ctypes.c_int]
     L.gg_testing_force_variant.restype = ctypes.c_int
     L.gg_version.restype = ctypes.c_int
+    L.gg_last_error.restype = ctypes.c_char_p
     _lib = L
     return L
 
@@ -168,7 +177,11 @@ def forward(A: torch.Tensor, W: torch.Tensor, offs: torch.Tensor, out: torch.Ten
     return out
 
 
-def _epilogue(bias, bias_scale, act, E, N):
+def _flags(zero_tail: bool, w_nk: bool) -> int:
+    return (FLAG_ZERO_TAIL if zero_tail else 0) | (FLAG_W_NK if w_nk else 0)
+
+
+def _epilogue(bias, bias_scale, act, E, N, flags=0):
     if bias is not None:
         _check(bias, "bias", torch.bfloat16, 2)
         if tuple(bias.shape) != (E, N):
@@ -177,30 +190,76 @@ def _epilogue(bias, bias_scale, act, E, N):
         _check(bias_scale, "bias_scale", torch.float32, 1)
     if act not in (ACT_NONE, ACT_SILU_MUL):
         raise ValueError("act must be ACT_NONE or ACT_SILU_MUL")
-    return _Epilogue(_ptr(bias), _ptr(bias_scale), act)
+    return _Epilogue(_ptr(bias), _ptr(bias_scale), act, flags)
 
 
 def forward_ex(A: torch.Tensor, W: torch.Tensor, offs: torch.Tensor, out: torch.Tensor, *,
                bias: Optional[torch.Tensor] = None, bias_scale: Optional[torch.Tensor] = None,
-               act: int = ACT_NONE, status: Optional[torch.Tensor] = None,
-               stream=None) -> torch.Tensor:
+               act: int = ACT_NONE, zero_tail: bool = False, w_nk: bool = False,
+               status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """Forward with a fused epilogue: h = A @ W[e] + bias_scale[r] * bias[e]; with
     act=ACT_SILU_MUL out = silu(gate) * up over gate/up column blocks of 128 (N % 256 == 0),
-    and out has N/2 columns. bias_scale is read only for rows inside a group."""
+    and out has N/2 columns. bias_scale is read only for rows inside a group. zero_tail
+    writes zeros to the rows past the last offset; w_nk takes W as [E, N, K]."""
     _check(A, "A", torch.bfloat16, 2)
     _check(W, "W", torch.bfloat16, 3)
     _check(offs, "offs", torch.int32, 1)
     _check(out, "out", torch.bfloat16, 2)
     rows, K = A.shape
-    E, K2, N = W.shape
+    if w_nk:
+        E, N, K2 = W.shape
+    else:
+        E, K2, N = W.shape
     ncols = N // 2 if act == ACT_SILU_MUL else N
     if K2 != K or offs.numel() != E or tuple(out.shape) != (rows, ncols):
         raise ValueError("shape mismatch: A[rows,K], W[E,K,N], offs[E], out[rows,N or N/2]")
-    epi = _epilogue(bias, bias_scale, act, E, N)
+    epi = _epilogue(bias, bias_scale, act, E, N, _flags(zero_tail, w_nk))
     rc = lib().gg_forward_ex(_ptr(A), _ptr(W), _ptr(offs), _ptr(out), rows, K, N, E,
                              ctypes.byref(epi), _status_ptr(status), _stream_handle(stream))
     _raise(rc, "gg_forward_ex")
     return out
+
+
+def dgrad_ex(dY: torch.Tensor, W: torch.Tensor, offs: torch.Tensor, dX: torch.Tensor, *,
+             zero_tail: bool = False, w_nk: bool = False, status: Optional[torch.Tensor] = None,
+             stream=None) -> torch.Tensor:
+    """dgrad with flags: zero_tail writes zeros to the rows past the last offset; w_nk takes
+    W as [E, N, K]."""
+    _check(dY, "dY", torch.bfloat16, 2)
+    _check(W, "W", torch.bfloat16, 3)
+    _check(offs, "offs", torch.int32, 1)
+    _check(dX, "dX", torch.bfloat16, 2)
+    rows, N = dY.shape
+    if w_nk:
+        E, N2, K = W.shape
+    else:
+        E, K, N2 = W.shape
+    if N2 != N or offs.numel() != E or tuple(dX.shape) != (rows, K):
+        raise ValueError("shape mismatch: dY[rows,N], W, offs[E], dX[rows,K]")
+    rc = lib().gg_dgrad_ex(_ptr(dY), _ptr(W), _ptr(offs), _ptr(dX), rows, K, N, E,
+                           _flags(zero_tail, w_nk), _status_ptr(status), _stream_handle(stream))
+    _raise(rc, "gg_dgrad_ex")
+    return dX
+
+
+def wgrad_ex(A: torch.Tensor, dY: torch.Tensor, offs: torch.Tensor, dW: torch.Tensor, *,
+             w_nk: bool = False, status: Optional[torch.Tensor] = None,
+             stream=None) -> torch.Tensor:
+    """wgrad with flags: w_nk writes dW as [E, N, K] (dW[e] = dY_e^T @ A_e)."""
+    _check(A, "A", torch.bfloat16, 2)
+    _check(dY, "dY", torch.bfloat16, 2)
+    _check(offs, "offs", torch.int32, 1)
+    _check(dW, "dW", torch.bfloat16, 3)
+    rows, K = A.shape
+    rows2, N = dY.shape
+    E = offs.numel()
+    want = (E, N, K) if w_nk else (E, K, N)
+    if rows2 != rows or tuple(dW.shape) != want:
+        raise ValueError(f"shape mismatch: dW must be {want}")
+    rc = lib().gg_wgrad_ex(_ptr(A), _ptr(dY), _ptr(offs), _ptr(dW), rows, K, N, E,
+                           _flags(False, w_nk), _status_ptr(status), _stream_handle(stream))
+    _raise(rc, "gg_wgrad_ex")
+    return dW
 
 
 def masked_forward_ex(A: torch.Tensor, W: torch.Tensor, masked_m: torch.Tensor,
@@ -343,16 +402,52 @@ def route(topk_ids: torch.Tensor, X: torch.Tensor, E: int, *,
     return A_packed, row_of, offs
 
 
+class _GroupedMM(torch.autograd.Function):
+    """out = grouped A @ W over the offsets; backward runs dgrad and wgrad on the same
+    groups. Output and input gradient are complete tensors (zero past the last offset)."""
+
+    @staticmethod
+    def forward(ctx, A, W, offs, w_nk):
+        N = W.shape[1] if w_nk else W.shape[2]
+        out = torch.empty((A.shape[0], N), dtype=A.dtype, device=A.device)
+        forward_ex(A, W, offs, out, zero_tail=True, w_nk=w_nk)
+        ctx.save_for_backward(A, W, offs)
+        ctx.w_nk = w_nk
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        A, W, offs = ctx.saved_tensors
+        dout = dout.contiguous()
+        dA = dW = None
+        if ctx.needs_input_grad[0]:
+            dA = torch.empty_like(A)
+            dgrad_ex(dout, W, offs, dA, zero_tail=True, w_nk=ctx.w_nk)
+        if ctx.needs_input_grad[1]:
+            dW = torch.empty_like(W)
+            wgrad_ex(A, dout, offs, dW, w_nk=ctx.w_nk)
+        return dA, dW, None, None
+
+
 def grouped_mm(A: torch.Tensor, W: torch.Tensor, offs: torch.Tensor,
-               out: Optional[torch.Tensor] = None, **kw) -> torch.Tensor:
-    """Forward with an optional caller-owned ``out`` (allocated uninitialised when None)."""
+               out: Optional[torch.Tensor] = None, *, w_nk: bool = False) -> torch.Tensor:
+    """``torch._grouped_mm(x, w, offs)``-style call (PyTorch issue 152668). With autograd
+    (A or W requiring grad) the backward runs gg_dgrad / gg_wgrad and rows past the last
+    offset are zero in the output and in dA. Without autograd, ``out`` may be given (rows
+    past the last offset are then left as they are)."""
+    if torch.is_grad_enabled() and (A.requires_grad or W.requires_grad):
+        if out is not None:
+            raise ValueError("out= cannot be used with autograd")
+        return _GroupedMM.apply(A, W, offs, w_nk)
     if out is None:
-        out = torch.empty((A.shape[0], W.shape[2]), dtype=A.dtype, device=A.device)
-    return forward(A, W, offs, out, **kw)
+        N = W.shape[1] if w_nk else W.shape[2]
+        out = torch.empty((A.shape[0], N), dtype=A.dtype, device=A.device)
+    return forward_ex(A, W, offs, out, w_nk=w_nk)
 
 
 __all__ = [
-    "forward", "forward_ex", "dgrad", "wgrad", "wgrad_f32", "masked_forward",
+    "forward", "forward_ex", "dgrad", "dgrad_ex", "wgrad", "wgrad_ex", "wgrad_f32",
+    "masked_forward", "FLAG_ZERO_TAIL", "FLAG_W_NK",
     "masked_forward_ex", "ACT_NONE", "ACT_SILU_MUL", "route", "route_workspace_bytes", "grouped_mm", "status_string", "version",
     "set_watchdog_ns", "testing_skip_first_load", "testing_force_variant", "lib", "GGError", "LIB_PATH",
     "DEV_BAD_OFFSETS", "DEV_BAD_MASKED_M", "DEV_TIMEOUT", "DEV_ERROR_MASK", "DEV_LAUNCHED",

@@ -3,6 +3,7 @@
 // synchronises or clears memory; everything is ordered on the caller's stream.
 #include <atomic>
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 
@@ -22,6 +23,14 @@ constexpr int kMaxDevices = 64;
 constexpr uint64_t kDefaultWatchdogNs = 4000000000ull;
 
 std::atomic<uint64_t> g_watchdog_ns{kDefaultWatchdogNs};
+
+// Text of the last failure in this thread (gg_last_error).
+thread_local char g_err[256] = "";
+
+gg_status cuda_fail(const char* where, cudaError_t e) {
+  snprintf(g_err, sizeof(g_err), "%s: %s", where, cudaGetErrorString(e));
+  return GG_ERR_CUDA;
+}
 std::atomic<int> g_skip_first_load{0};
 std::atomic<int> g_force_variant{0};  // test hook: 0 automatic, 1 single CTA, 2 CTA pair
 
@@ -55,16 +64,20 @@ std::mutex g_dev_mu;
 
 gg_status device_info(DeviceInfo* out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return GG_ERR_CUDA;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
   if (dev < 0 || dev >= kMaxDevices) return GG_ERR_UNSUPPORTED;
+  // Tensor maps are encoded with a driver call, which needs a current context; a thread
+  // that has not touched CUDA yet (e.g. an autograd worker) may have none.
+  if ((e = cudaSetDevice(dev)) != cudaSuccess) return cuda_fail("cudaSetDevice", e);
   std::lock_guard<std::mutex> lk(g_dev_mu);
   DeviceInfo& d = g_dev[dev];
   if (!d.ready) {
     int major = 0, minor = 0, sms = 0;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return GG_ERR_CUDA;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail("cudaDeviceGetAttribute", e);
     d.sms = sms;
     d.sm100 = (major == 10 && minor == 0);
     d.ready = true;
@@ -79,7 +92,10 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
               const uint64_t* strides_bytes, const uint32_t* box) {
   auto fn = encode_fn();
-  if (fn == nullptr) return false;
+  if (fn == nullptr) {
+    snprintf(g_err, sizeof(g_err), "cuTensorMapEncodeTiled: driver entry point not found");
+    return false;
+  }
   cuuint64_t gdim[4];
   cuuint64_t gstr[3];
   cuuint32_t bdim[4];
@@ -94,6 +110,8 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
                   gdim, gstr, bdim, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    snprintf(g_err, sizeof(g_err), "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
   return r == CUDA_SUCCESS;
 }
 
@@ -144,7 +162,8 @@ gg_status launch(const CUtensorMap& a, const CUtensorMap& b, const gg::Params& p
   using L = gg::Layout<BN, STAGES, PAIR>;
   const size_t smem = L::bytes(p.E);
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return GG_ERR_CUDA;
+  cudaError_t ce = cudaGetDevice(&dev);
+  if (ce != cudaSuccess) return cuda_fail("cudaGetDevice", ce);
   static bool attr_done[kMaxDevices] = {};
   static int max_units[kMaxDevices] = {};
   static std::mutex mu;
@@ -152,9 +171,9 @@ gg_status launch(const CUtensorMap& a, const CUtensorMap& b, const gg::Params& p
     std::lock_guard<std::mutex> lk(mu);
     if (!attr_done[dev]) {
       const int max_smem = (int)L::bytes(GG_MAX_EXPERTS);
-      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) !=
-          cudaSuccess)
-        return GG_ERR_CUDA;
+      if ((ce = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     max_smem)) != cudaSuccess)
+        return cuda_fail("cudaFuncSetAttribute", ce);
       int units = di.sms;
       if (PAIR) {
         // persistent grid: as many CTA pairs as can be resident at once
@@ -170,8 +189,9 @@ gg_status launch(const CUtensorMap& a, const CUtensorMap& b, const gg::Params& p
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int clusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1)
-          return GG_ERR_CUDA;
+        if ((ce = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg)) != cudaSuccess)
+          return cuda_fail("cudaOccupancyMaxActiveClusters", ce);
+        if (clusters < 1) return cuda_fail("cudaOccupancyMaxActiveClusters", cudaErrorUnknown);
         units = clusters;
       }
       max_units[dev] = units;
@@ -182,7 +202,8 @@ gg_status launch(const CUtensorMap& a, const CUtensorMap& b, const gg::Params& p
   if (units < 1) units = 1;
   if (!PAIR) {
     kern<<<(unsigned)units, gg::NUM_THREADS, smem, stream>>>(a, b, p);
-    return cudaGetLastError() == cudaSuccess ? GG_OK : GG_ERR_CUDA;
+    ce = cudaGetLastError();
+    return ce == cudaSuccess ? GG_OK : cuda_fail("kernel launch", ce);
   }
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -196,8 +217,10 @@ gg_status launch(const CUtensorMap& a, const CUtensorMap& b, const gg::Params& p
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, a, b, p) != cudaSuccess) return GG_ERR_CUDA;
-  return cudaGetLastError() == cudaSuccess ? GG_OK : GG_ERR_CUDA;
+  if ((ce = cudaLaunchKernelEx(&cfg, kern, a, b, p)) != cudaSuccess)
+    return cuda_fail("cudaLaunchKernelEx", ce);
+  ce = cudaGetLastError();
+  return ce == cudaSuccess ? GG_OK : cuda_fail("kernel launch", ce);
 }
 
 gg::Params base_params(const int32_t* groups, void* out, int32_t* status, int64_t rows_alloc,
@@ -314,6 +337,8 @@ gg_status set_epilogue(gg::Params* p, const gg_epilogue* epi, int64_t N) {
   return GG_OK;
 }
 
+// Forward, out = A . W[e] (+ epilogue). W is [E, K, N] (MN-major B: the forward pipeline)
+// or, with GG_FLAG_W_NK, [E, N, K] (K-major B: the pipeline of dgrad).
 gg_status forward_impl(const void* A, const void* W, const int32_t* offs, void* out,
                        int64_t rows_alloc, int64_t K, int64_t N, int32_t E,
                        const gg_epilogue* epi, int32_t* dev_status, cudaStream_t stream) {
@@ -324,31 +349,89 @@ gg_status forward_impl(const void* A, const void* W, const int32_t* offs, void* 
   if (rows_alloc == 0) return GG_OK;  // no row can belong to a group
   if (A == nullptr || out == nullptr) return GG_ERR_INVALID_ARG;
   if (!aligned16(A) || !aligned16(W) || !aligned16(out)) return GG_ERR_UNSUPPORTED;
+  const int32_t flags = epi != nullptr ? epi->flags : 0;
+  if (flags & ~(GG_FLAG_ZERO_TAIL | GG_FLAG_W_NK)) return GG_ERR_INVALID_ARG;
   const bool silu = epi != nullptr && epi->act == GG_ACT_SILU_MUL;
+  const bool wnk = (flags & GG_FLAG_W_NK) != 0;
   const bool pair = use_pair(rows_alloc, E);
   const bool chunked = (N % 64) == 0;
   const uint32_t bcols = pair ? kBN / 2 : kBN;
   CUtensorMap ma, mb;
   if (!map_2d(&ma, A, rows_alloc, K, 64, gg::BM)) return GG_ERR_CUDA;
-  if (chunked ? !map_w_chunked(&mb, W, E, K, N, 64, bcols / 64) : !map_w(&mb, W, E, K, N, 64, 64))
+  if (wnk) {
+    // W[e] is [N, K]: K-major B, one box of bcols rows of N per stage
+    if (!map_w(&mb, W, E, N, K, 64, bcols)) return GG_ERR_CUDA;
+  } else if (chunked ? !map_w_chunked(&mb, W, E, K, N, 64, bcols / 64)
+                     : !map_w(&mb, W, E, K, N, 64, 64)) {
     return GG_ERR_CUDA;
+  }
   gg::Params p = base_params(offs, out, dev_status, rows_alloc, E);
   p.red_len = (int32_t)K;
-  p.b_chunked = chunked ? 1 : 0;
+  p.b_chunked = (!wnk && chunked) ? 1 : 0;
+  p.zero_tail = (flags & GG_FLAG_ZERO_TAIL) ? 1 : 0;
   if ((s = set_epilogue(&p, epi, N)) != GG_OK) return s;
   const int64_t out_cols = silu ? N / 2 : N;
   p.out_cols = (int32_t)out_cols;
   p.prod_cols = (int32_t)N;
   set_store_width(&p, out, out_cols);
+  const int64_t tiles = (cdiv(rows_alloc, (pair ? 2 : 1) * gg::BM) + E + 1) * cdiv(N, kBN);
+  if (wnk) {
+    if (pair) {
+      if (silu) return launch<Mode::Dgrad, kBN, kPairStages, true, false, 1>(ma, mb, p, tiles, di, stream);
+      return launch<Mode::Dgrad, kBN, kPairStages, true>(ma, mb, p, tiles, di, stream);
+    }
+    if (silu) return launch<Mode::Dgrad, kBN, kStages, false, false, 1>(ma, mb, p, tiles, di, stream);
+    return launch<Mode::Dgrad, kBN, kStages, false>(ma, mb, p, tiles, di, stream);
+  }
   if (pair) {
-    const int64_t tiles = (cdiv(rows_alloc, 2 * gg::BM) + E) * cdiv(N, kBN);
-    if (silu)
-      return launch<Mode::Forward, kBN, kPairStages, true, false, 1>(ma, mb, p, tiles, di, stream);
+    if (silu) return launch<Mode::Forward, kBN, kPairStages, true, false, 1>(ma, mb, p, tiles, di, stream);
     return launch<Mode::Forward, kBN, kPairStages, true>(ma, mb, p, tiles, di, stream);
   }
-  const int64_t tiles = (cdiv(rows_alloc, gg::BM) + E) * cdiv(N, kBN);
   if (silu) return launch<Mode::Forward, kBN, kStages, false, false, 1>(ma, mb, p, tiles, di, stream);
   return launch<Mode::Forward, kBN, kStages, false>(ma, mb, p, tiles, di, stream);
+}
+
+// dgrad, dX = dY . W[e]^T. W is [E, K, N] (K-major B: the dgrad pipeline) or, with
+// GG_FLAG_W_NK, [E, N, K] (MN-major B: the pipeline of the forward).
+gg_status dgrad_impl(const void* dY, const void* W, const int32_t* offs, void* dX,
+                     int64_t rows_alloc, int64_t K, int64_t N, int32_t E, int32_t flags,
+                     int32_t* dev_status, cudaStream_t stream) {
+  DeviceInfo di;
+  gg_status s = check_common(rows_alloc, K, N, E, offs, dev_status, &di);
+  if (s != GG_OK) return s;
+  if (flags & ~(GG_FLAG_ZERO_TAIL | GG_FLAG_W_NK)) return GG_ERR_INVALID_ARG;
+  if (W == nullptr) return GG_ERR_INVALID_ARG;
+  if (rows_alloc == 0) return GG_OK;
+  if (dY == nullptr || dX == nullptr) return GG_ERR_INVALID_ARG;
+  if (!aligned16(dY) || !aligned16(W) || !aligned16(dX)) return GG_ERR_UNSUPPORTED;
+  const bool wnk = (flags & GG_FLAG_W_NK) != 0;
+  const bool pair = use_pair(rows_alloc, E);
+  const uint32_t bcols = pair ? kBN / 2 : kBN;
+  const bool chunked = (K % 64) == 0;
+  CUtensorMap ma, mb;
+  if (!map_2d(&ma, dY, rows_alloc, N, 64, gg::BM)) return GG_ERR_CUDA;
+  if (wnk) {
+    // W[e] is [N, K] with the output dimension K contiguous: MN-major B over (K, N)
+    if (chunked ? !map_w_chunked(&mb, W, E, N, K, 64, bcols / 64)
+                : !map_w(&mb, W, E, N, K, 64, 64))
+      return GG_ERR_CUDA;
+  } else if (!map_w(&mb, W, E, K, N, 64, bcols)) {
+    return GG_ERR_CUDA;
+  }
+  gg::Params p = base_params(offs, dX, dev_status, rows_alloc, E);
+  p.red_len = (int32_t)N;
+  p.out_cols = (int32_t)K;
+  p.prod_cols = (int32_t)K;
+  p.b_chunked = (wnk && chunked) ? 1 : 0;
+  p.zero_tail = (flags & GG_FLAG_ZERO_TAIL) ? 1 : 0;
+  set_store_width(&p, dX, K);
+  const int64_t tiles = (cdiv(rows_alloc, (pair ? 2 : 1) * gg::BM) + E + 1) * cdiv(K, kBN);
+  if (wnk) {
+    if (pair) return launch<Mode::Forward, kBN, kPairStages, true>(ma, mb, p, tiles, di, stream);
+    return launch<Mode::Forward, kBN, kStages, false>(ma, mb, p, tiles, di, stream);
+  }
+  if (pair) return launch<Mode::Dgrad, kBN, kPairStages, true>(ma, mb, p, tiles, di, stream);
+  return launch<Mode::Dgrad, kBN, kStages, false>(ma, mb, p, tiles, di, stream);
 }
 
 gg_status masked_impl(const void* A, const void* W, const int32_t* masked_m, void* out,
@@ -420,34 +503,27 @@ gg_status gg_masked_forward_ex(const void* A, const void* W, const int32_t* mask
 gg_status gg_dgrad(const void* dY, const void* W, const int32_t* offs, void* dX,
                    int64_t rows_alloc, int64_t K, int64_t N, int32_t E, int32_t* dev_status,
                    cudaStream_t stream) {
-  DeviceInfo di;
-  gg_status s = check_common(rows_alloc, K, N, E, offs, dev_status, &di);
-  if (s != GG_OK) return s;
-  if (W == nullptr) return GG_ERR_INVALID_ARG;
-  if (rows_alloc == 0) return GG_OK;
-  if (dY == nullptr || dX == nullptr) return GG_ERR_INVALID_ARG;
-  if (!aligned16(dY) || !aligned16(W) || !aligned16(dX)) return GG_ERR_UNSUPPORTED;
-  CUtensorMap ma, mb;
-  const bool pair = use_pair(rows_alloc, E);
-  if (!map_2d(&ma, dY, rows_alloc, N, 64, gg::BM) ||
-      !map_w(&mb, W, E, K, N, 64, pair ? kBN / 2 : kBN))
-    return GG_ERR_CUDA;
-  gg::Params p = base_params(offs, dX, dev_status, rows_alloc, E);
-  p.red_len = (int32_t)N;
-  p.out_cols = (int32_t)K;
-  p.prod_cols = (int32_t)K;
-  set_store_width(&p, dX, K);
-  if (pair) {
-    const int64_t tiles = (cdiv(rows_alloc, 2 * gg::BM) + E) * cdiv(K, kBN);
-    return launch<Mode::Dgrad, kBN, kPairStages, true>(ma, mb, p, tiles, di, stream);
-  }
-  const int64_t tiles = (cdiv(rows_alloc, gg::BM) + E) * cdiv(K, kBN);
-  return launch<Mode::Dgrad, kBN, kStages, false>(ma, mb, p, tiles, di, stream);
+  return dgrad_impl(dY, W, offs, dX, rows_alloc, K, N, E, 0, dev_status, stream);
+}
+
+gg_status gg_dgrad_ex(const void* dY, const void* W, const int32_t* offs, void* dX,
+                      int64_t rows_alloc, int64_t K, int64_t N, int32_t E, int32_t flags,
+                      int32_t* dev_status, cudaStream_t stream) {
+  return dgrad_impl(dY, W, offs, dX, rows_alloc, K, N, E, flags, dev_status, stream);
 }
 
 gg_status gg_wgrad(const void* A, const void* dY, const int32_t* offs, void* dW,
                    int64_t rows_alloc, int64_t K, int64_t N, int32_t E, int32_t* dev_status,
                    cudaStream_t stream) {
+  return wgrad_impl(A, dY, offs, dW, false, 1.f, 0.f, rows_alloc, K, N, E, dev_status, stream);
+}
+
+gg_status gg_wgrad_ex(const void* A, const void* dY, const int32_t* offs, void* dW,
+                      int64_t rows_alloc, int64_t K, int64_t N, int32_t E, int32_t flags,
+                      int32_t* dev_status, cudaStream_t stream) {
+  if (flags & ~GG_FLAG_W_NK) return GG_ERR_INVALID_ARG;
+  if (flags & GG_FLAG_W_NK)  // dW[e] = dY_e^T A_e, stored [E, N, K]
+    return wgrad_impl(dY, A, offs, dW, false, 1.f, 0.f, rows_alloc, N, K, E, dev_status, stream);
   return wgrad_impl(A, dY, offs, dW, false, 1.f, 0.f, rows_alloc, K, N, E, dev_status, stream);
 }
 
@@ -483,5 +559,7 @@ int gg_testing_force_variant(int variant) {
 }
 
 int gg_version(void) { return 100; }
+
+const char* gg_last_error(void) { return g_err; }
 
 }  // extern "C"

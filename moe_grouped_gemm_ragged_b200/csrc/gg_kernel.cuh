@@ -119,6 +119,9 @@ struct Params {
   const __nv_bfloat16* bias;
   const float* bias_scale;
   int32_t bias_ld;
+  // forward/dgrad: rows at and past the last effective offset are written with zeros (a
+  // pseudo-group after the last expert whose tiles have no reduction stages)
+  int32_t zero_tail;
 };
 
 template <int BN, int STAGES, bool PAIR>
@@ -135,9 +138,9 @@ struct Layout {
   static constexpr uint32_t OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr uint32_t OFF_TAB = OFF_MISC + 16;
   static constexpr uint32_t TMEM_COLS = 2 * BN;
-  // gstart[E], gend[E], prefix[E+1], order[E] (int32)
+  // gstart[E+1], gend[E+1], prefix[E+2], order[E] (int32); group E is the zero tail
   static __host__ __device__ constexpr uint32_t bytes(int E) {
-    return OFF_TAB + 4u * (4u * (uint32_t)E + 1u) + 1024u /* alignment slack */;
+    return OFF_TAB + 4u * (4u * ((uint32_t)E + 1u) + 1u) + 1024u /* alignment slack */;
   }
 };
 
@@ -284,6 +287,13 @@ __device__ void build_table(const Params& p, const Shared& sh) {
     if constexpr (MODE == Mode::Wgrad) {
       const int32_t KT = (p.wg_K + TM - 1) / TM;
       *sh.total = E * KT * NT;
+    } else if (MODE != Mode::Masked && p.zero_tail) {
+      // rows [t'_{E-1}, rows_alloc): one more group, of zero tiles
+      const int32_t tail = (int32_t)(p.rows_alloc - prev_end);
+      sh.gstart[E] = prev_end;
+      sh.gend[E] = (int32_t)p.rows_alloc;
+      sh.prefix[E + 1] = tiles_carry + ((tail + TM - 1) / TM) * NT;
+      *sh.total = sh.prefix[E + 1];
     } else {
       *sh.total = tiles_carry;
     }
@@ -327,8 +337,8 @@ __device__ __forceinline__ Tile decode_tile(int32_t t, const Params& p, const Sh
     tl.row_end = (int64_t)e * p.wg_K + p.wg_K;
     tl.a_row0 = 0;
   } else {
-    // largest e with prefix[e] <= t
-    int32_t lo = 0, hi = p.E - 1;
+    // largest e with prefix[e] <= t (group E is the zero tail, when present)
+    int32_t lo = 0, hi = (MODE != Mode::Masked && p.zero_tail) ? p.E : p.E - 1;
     while (lo < hi) {
       const int32_t mid = (lo + hi + 1) >> 1;
       if (sh.prefix[mid] <= t) lo = mid; else hi = mid - 1;
@@ -342,7 +352,7 @@ __device__ __forceinline__ Tile decode_tile(int32_t t, const Params& p, const Sh
     tl.row0 = tl.a_row0;
     tl.row_end = sh.gend[e];
     tl.n0 = nt * BN;
-    tl.kblocks = (p.red_len + BK - 1) / BK;
+    tl.kblocks = e < p.E ? (p.red_len + BK - 1) / BK : 0;
     tl.k0 = 0;
     tl.tok0 = 0;
     tl.tok_len = 0;
@@ -389,9 +399,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   sh.total = reinterpret_cast<int32_t*>(smem + L::OFF_MISC + 8);
   int32_t* tab = reinterpret_cast<int32_t*>(smem + L::OFF_TAB);
   sh.gstart = tab;
-  sh.gend = tab + p.E;
-  sh.prefix = tab + 2 * p.E;
-  sh.order = tab + 3 * p.E + 1;
+  sh.gend = tab + (p.E + 1);
+  sh.prefix = tab + 2 * (p.E + 1);
+  sh.order = tab + 3 * (p.E + 1) + 1;
 
   const uint32_t warp = threadIdx.x / 32;
   const uint32_t lane = ptx::lane_id();
@@ -721,8 +731,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               }
             }
           } else {
-            for (int c = 0; c < CW; c += 8) {
-              const int32_t col = col0 + c;
+            // SiLU-and-mul halves the columns: this warp's outputs start at half its offset
+            const int32_t zc0 = ACT == 1 ? tl.n0 / 2 + c_off / 2 : col0;
+            const int32_t zcw = ACT == 1 ? CW / 2 : CW;
+            for (int c = 0; c < zcw; c += 8) {
+              const int32_t col = zc0 + c;
               if (col < p.out_cols)
                 *reinterpret_cast<uint4*>(orow_ptr + col) = make_uint4(0u, 0u, 0u, 0u);
             }
