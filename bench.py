@@ -16,7 +16,6 @@ times the CPU oracle on a bounded sample of the same workload (rank 0 only).
 from __future__ import annotations
 
 import argparse
-import glob
 import hashlib
 import json
 import os
@@ -40,18 +39,23 @@ UNIT = "TFLOP/s"
 #   --clock-control none -k regex:grouped_gemm -s 12 -c 4 python bench.py --steps 1 --warmup 3
 #   --no-e2e --no-cpu   (see profiles/grouped_gemm_large_launch_list.md)
 NCU_TRAFFIC = {
-    ("forward", "large"): 23.285e9,
-    ("dgrad", "large"): 18.401e9,
-    ("wgrad", "large"): 14.635e9,
+    ("forward", "large"): 12.376e9,
+    ("dgrad", "large"): 11.844e9,
+    ("wgrad", "large"): 14.618e9,
     ("masked", "large"): 0.023e9,
 }
-NCU_TRAFFIC_SRC_HASH = "935250cbfbbd458b"
+NCU_TRAFFIC_SRC_HASH = "cb440b395283ee9a"
+
+
+GEMM_SOURCES = ("gg_kernel.cuh", "ptx.cuh", "gg_api.cu")  # the grouped GEMM kernels + launch
 
 
 def kernel_source_hash() -> str:
+    """Hash of the sources of the grouped GEMM kernels: the stored ncu traffic is reported
+    only while it matches (a changed kernel invalidates the counters)."""
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "moe_grouped_gemm_ragged_b200", "csrc", "*"))):
-        h.update(open(f, "rb").read())
+    for f in GEMM_SOURCES:
+        h.update(open(os.path.join(ROOT, "moe_grouped_gemm_ragged_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -429,19 +433,22 @@ def run_e2e(args, gg, r, m, dev, stream, ws, barrier):
     hdX = torch.empty(dX.shape, dtype=dX.dtype).pin_memory()
     hdW = torch.empty(dW.shape, dtype=dW.dtype).pin_memory()
     hmout = torch.empty(mout.shape, dtype=mout.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (hA, hW, hdY, hoffs, hmA, hmW, hmm))
-    d2h = sum(t.numel() * t.element_size() for t in (hout, hdX, hdW, hmout))
+    # bytes the step moves: the rows inside the groups (T of them), all of W and dW, offsets
+    T = r.T
+    nb = lambda t: t.numel() * t.element_size()
+    h2d = (T * (K + N) * 2 + nb(hW) + nb(hoffs) + nb(hmA) + nb(hmW) + nb(hmm))
+    d2h = T * (N + K) * 2 + nb(hdW) + nb(hmout)
+
+    staging = {"A": dA, "W": dWt, "dY": ddY, "offs": doffs, "out": out, "dX": dX, "dW": dW}
 
     def step():
-        for d, h in ((dA, hA), (dWt, hW), (ddY, hdY), (doffs, hoffs), (dmA, hmA), (dmW, hmW),
-                     (dmm, hmm)):
+        # the ragged passes through the host-buffer entry point (expert chunks, copies both
+        # ways overlapped with the GEMMs), then the masked call with its own copies
+        gg.layer_step_host(hA, hW, hdY, hoffs, hout, hdX, hdW, staging, chunks=args.e2e_chunks)
+        for d, h in ((dmA, hmA), (dmW, hmW), (dmm, hmm)):
             d.copy_(h, non_blocking=True)
-        gg.forward(dA, dWt, doffs, out)
-        gg.dgrad(ddY, dWt, doffs, dX)
-        gg.wgrad(dA, ddY, doffs, dW)
         gg.masked_forward(dmA, dmW, dmm, mout)
-        for h, d in ((hout, out), (hdX, dX), (hdW, dW), (hmout, mout)):
-            h.copy_(d, non_blocking=True)
+        hmout.copy_(mout, non_blocking=True)
 
     step()
     torch.cuda.synchronize()
@@ -457,7 +464,9 @@ def run_e2e(args, gg, r, m, dev, stream, ws, barrier):
     ms = reduce_max(e0.elapsed_time(e1) / steps, dev)
     flops = 3 * r.flops + m.flops
     return {"value": ws * flops / (ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms,
-            "steps": steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "steps": steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "api": "gg_layer_step_host + gg_masked_forward",
+            "expert_chunks": args.e2e_chunks or 8}
 
 
 def main(argv=None):
@@ -469,6 +478,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="large",
                     choices=["large", "large_unaligned", "gateup", "downproj", "large_e2"])
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-chunks", type=int, default=0,
+                    help="expert chunks of the host-buffer pass (0: the library default)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-extras", action="store_true")

@@ -243,6 +243,35 @@ GG_API gg_status gg_route_noalloc(const int32_t* topk_ids, int64_t T_tok, int32_
                                   int32_t* offs, int32_t* dev_status, cudaStream_t stream);
 
 /* A static, human-readable name for a status. */
+/*
+ * One forward + backward pass of the grouped GEMM layer on operands in HOST memory:
+ *   out = forward(A, W, offs), dX = dgrad(dY, W, offs), dW = wgrad(A, dY, offs),
+ * the same three definitions as gg_forward / gg_dgrad / gg_wgrad, streamed through the GPU in
+ * chunks of consecutive experts: while one chunk computes on `stream`, the next chunk's
+ * operands are copied host -> device and the previous chunk's results device -> host, on two
+ * copy streams that the library creates once per device and keeps.
+ *   host (pinned, or the copies do not overlap): A_h bf16 [rows, K], W_h bf16 [E, K, N],
+ *     dY_h bf16 [rows, N], offs_h int32 [E] cumulative end offsets; results out_h
+ *     [rows, N], dX_h [rows, K], dW_h [E, K, N]; rows >= offs_h[E-1] of out_h / dX_h are
+ *     not written.
+ *   device staging, caller-owned, the same shapes: A_d, W_d, dY_d, out_d, dX_d, dW_d, and
+ *     offs_d int32 [E], which ends up holding chunk-relative offsets.
+ *   chunks: number of expert chunks (0: 8; at most E and 32).
+ * The offsets are host data here and are checked on the host: non-decreasing within
+ * [0, rows], else GG_ERR_INVALID_ARG and nothing is enqueued. The call returns once all work
+ * is enqueued; `stream` is ordered after the last copy back, so the host results are valid
+ * once `stream` is synchronised, and the work starts after what `stream` held before the
+ * call. Calls from several threads are serialised while they enqueue. Not for stream capture.
+ * The pages have no counterpart: this is the host-buffer form of the three passes, with the
+ * host link overlapped with the GEMMs.
+ */
+GG_API gg_status gg_layer_step_host(const void* A_h, const void* W_h, const void* dY_h,
+                                    const int32_t* offs_h, void* out_h, void* dX_h,
+                                    void* dW_h, void* A_d, void* W_d, void* dY_d,
+                                    int32_t* offs_d, void* out_d, void* dX_d, void* dW_d,
+                                    int64_t rows, int64_t K, int64_t N, int32_t E,
+                                    int32_t chunks, int32_t* dev_status, cudaStream_t stream);
+
 GG_API const char* gg_status_string(gg_status s);
 
 /* Watchdog bound of every in-kernel wait, in nanoseconds, for later calls from any

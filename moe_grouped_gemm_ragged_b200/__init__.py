@@ -84,6 +84,8 @@ def lib() -> ctypes.CDLL:
     L.gg_route_workspace_bytes.restype = ctypes.c_size_t
     L.gg_route.argtypes = [P, i64, i32, i32, P, i64, P, P, P, P, ctypes.c_size_t, P, P]
     L.gg_route.restype = ctypes.c_int
+    L.gg_layer_step_host.argtypes = [P] * 14 + [i64, i64, i64, i32, i32, P, P]
+    L.gg_layer_step_host.restype = ctypes.c_int
     L.gg_status_string.argtypes = [ctypes.c_int]
     L.gg_status_string.restype = ctypes.c_char_p
     L.gg_set_watchdog_ns.argtypes = [ctypes.c_uint64]
@@ -366,6 +368,57 @@ def masked_forward(A: torch.Tensor, W: torch.Tensor, masked_m: torch.Tensor,
     return out
 
 
+def _check_host(t: torch.Tensor, name: str, dtype, ndim: int):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cpu":
+        raise ValueError(f"{name} must be a host tensor")
+    if t.dtype != dtype or t.dim() != ndim or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {ndim}-d {dtype} tensor")
+
+
+def layer_step_host(A_h: torch.Tensor, W_h: torch.Tensor, dY_h: torch.Tensor,
+                    offs_h: torch.Tensor, out_h: torch.Tensor, dX_h: torch.Tensor,
+                    dW_h: torch.Tensor, staging: dict, *, chunks: int = 0,
+                    status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Forward + backward of the grouped GEMM layer on host tensors (``gg_layer_step_host``):
+    out_h = forward(A_h, W_h), dX_h = dgrad(dY_h, W_h), dW_h = wgrad(A_h, dY_h), streamed
+    through the GPU by expert chunks with the copies overlapped with the GEMMs.
+
+    Host tensors (pin them for overlap): A_h bf16 [rows, K], W_h bf16 [E, K, N], dY_h bf16
+    [rows, N], offs_h int32 [E]; results out_h [rows, N], dX_h [rows, K], dW_h [E, K, N].
+    ``staging`` holds caller-owned CUDA tensors of the same shapes under the keys
+    ``A, W, dY, offs, out, dX, dW``. Returns once enqueued on ``stream`` (default: the
+    current stream); synchronise it before reading the host results."""
+    for t, n, d, k in ((A_h, "A_h", torch.bfloat16, 2), (W_h, "W_h", torch.bfloat16, 3),
+                       (dY_h, "dY_h", torch.bfloat16, 2), (offs_h, "offs_h", torch.int32, 1),
+                       (out_h, "out_h", torch.bfloat16, 2), (dX_h, "dX_h", torch.bfloat16, 2),
+                       (dW_h, "dW_h", torch.bfloat16, 3)):
+        _check_host(t, n, d, k)
+    host = {"A": A_h, "W": W_h, "dY": dY_h, "offs": offs_h, "out": out_h, "dX": dX_h,
+            "dW": dW_h}
+    for k, h in host.items():
+        if k not in staging:
+            raise ValueError(f"staging['{k}'] is missing")
+        _check(staging[k], f"staging['{k}']", h.dtype, h.dim())
+        if staging[k].shape != h.shape:
+            raise ValueError(f"staging['{k}'] must have the shape {tuple(h.shape)}")
+    rows, K = A_h.shape
+    E, K2, N = W_h.shape
+    if (K2 != K or tuple(dY_h.shape) != (rows, N) or offs_h.numel() != E
+            or tuple(out_h.shape) != (rows, N) or tuple(dX_h.shape) != (rows, K)
+            or tuple(dW_h.shape) != (E, K, N)):
+        raise ValueError("shape mismatch: A[rows,K], W[E,K,N], dY[rows,N], offs[E], "
+                         "out[rows,N], dX[rows,K], dW[E,K,N]")
+    st = staging
+    rc = lib().gg_layer_step_host(
+        _ptr(A_h), _ptr(W_h), _ptr(dY_h), _ptr(offs_h), _ptr(out_h), _ptr(dX_h), _ptr(dW_h),
+        _ptr(st["A"]), _ptr(st["W"]), _ptr(st["dY"]), _ptr(st["offs"]), _ptr(st["out"]),
+        _ptr(st["dX"]), _ptr(st["dW"]), rows, K, N, E, int(chunks), _status_ptr(status),
+        _stream_handle(stream))
+    _raise(rc, "gg_layer_step_host")
+
+
 def route_workspace_bytes(n_assign: int, E: int) -> int:
     return int(lib().gg_route_workspace_bytes(int(n_assign), int(E)))
 
@@ -448,8 +501,10 @@ def grouped_mm(A: torch.Tensor, W: torch.Tensor, offs: torch.Tensor,
 __all__ = [
     "forward", "forward_ex", "dgrad", "dgrad_ex", "wgrad", "wgrad_ex", "wgrad_f32",
     "masked_forward", "FLAG_ZERO_TAIL", "FLAG_W_NK",
-    "masked_forward_ex", "ACT_NONE", "ACT_SILU_MUL", "route", "route_workspace_bytes", "grouped_mm", "status_string", "version",
-    "set_watchdog_ns", "testing_skip_first_load", "testing_force_variant", "lib", "GGError", "LIB_PATH",
+    "masked_forward_ex", "ACT_NONE", "ACT_SILU_MUL", "route", "route_workspace_bytes",
+    "grouped_mm", "layer_step_host", "status_string", "version",
+    "set_watchdog_ns", "testing_skip_first_load", "testing_force_variant", "lib", "GGError",
+    "LIB_PATH",
     "DEV_BAD_OFFSETS", "DEV_BAD_MASKED_M", "DEV_TIMEOUT", "DEV_ERROR_MASK", "DEV_LAUNCHED",
     "MAX_EXPERTS",
 ]

@@ -764,6 +764,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           ptx::tmem_ld_wait();
           const int32_t col = oc + c;  // output column of rg[0]
           if (row_ok && col < p.out_cols) {
+            if (bias_e != nullptr) {
+              // gate and up biases of these 32 columns, 8 at a time (16-byte loads)
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const uint4 bg = __ldg(reinterpret_cast<const uint4*>(bias_e + tl.n0 + half + c + 8 * j));
+                const uint4 bu =
+                    __ldg(reinterpret_cast<const uint4*>(bias_e + tl.n0 + BN / 2 + half + c + 8 * j));
+                const __nv_bfloat16* g8 = reinterpret_cast<const __nv_bfloat16*>(&bg);
+                const __nv_bfloat16* u8 = reinterpret_cast<const __nv_bfloat16*>(&bu);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                  rg[8 * j + u] = __float_as_uint(
+                      fmaf(s_row, __bfloat162float(g8[u]), __uint_as_float(rg[8 * j + u])));
+                  ru[8 * j + u] = __float_as_uint(
+                      fmaf(s_row, __bfloat162float(u8[u]), __uint_as_float(ru[8 * j + u])));
+                }
+              }
+            }
             uint32_t packed[16];
 #pragma unroll
             for (int h = 0; h < 16; ++h) {
@@ -771,11 +789,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
               for (int u = 0; u < 2; ++u) {
                 const int i = 2 * h + u;
-                float g = __uint_as_float(rg[i]), up = __uint_as_float(ru[i]);
-                if (bias_e != nullptr) {
-                  g = fmaf(s_row, __bfloat162float(bias_e[tl.n0 + half + c + i]), g);
-                  up = fmaf(s_row, __bfloat162float(bias_e[tl.n0 + BN / 2 + half + c + i]), up);
-                }
+                const float g = __uint_as_float(rg[i]), up = __uint_as_float(ru[i]);
                 v2[u] = g / (1.f + __expf(-g)) * up;
               }
               __nv_bfloat162 b2 = __floats2bfloat162_rn(v2[0], v2[1]);
@@ -805,8 +819,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ptx::tmem_ld_wait();
         if (c + 32 < CW) ptx::tmem_ld_32x32b_x32(taddr + c + 32, nxt);
         if (F32 && row_ok) {
-          // fp32 out = alpha * acc + beta * out; the old value is read only when beta != 0
+          // fp32 out = alpha * acc + beta * out; the old value is read only when beta != 0.
+          // All of the chunk's old values are loaded before the first store, so that the
+          // loads overlap instead of waiting behind stores the compiler cannot disambiguate.
           float* orow_f = p.out_f32 + orow * (int64_t)p.out_cols;
+          float4 old[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) old[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (p.beta != 0.f) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              if (col0 + c + j * 4 < p.out_cols)
+                old[j] = __ldg(reinterpret_cast<const float4*>(orow_f + col0 + c + j * 4));
+          }
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const int32_t col = col0 + c + j * 4;
@@ -816,11 +841,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                      p.alpha * __uint_as_float(cur[4 * j + 2]),
                                      p.alpha * __uint_as_float(cur[4 * j + 3]));
               if (p.beta != 0.f) {
-                const float4 o = *reinterpret_cast<const float4*>(orow_f + col);
-                v.x = fmaf(p.beta, o.x, v.x);
-                v.y = fmaf(p.beta, o.y, v.y);
-                v.z = fmaf(p.beta, o.z, v.z);
-                v.w = fmaf(p.beta, o.w, v.w);
+                v.x = fmaf(p.beta, old[j].x, v.x);
+                v.y = fmaf(p.beta, old[j].y, v.y);
+                v.z = fmaf(p.beta, old[j].z, v.z);
+                v.w = fmaf(p.beta, old[j].w, v.w);
               }
               *reinterpret_cast<float4*>(orow_f + col) = v;
             }

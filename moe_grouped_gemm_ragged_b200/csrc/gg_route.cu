@@ -40,17 +40,38 @@ __global__ void __launch_bounds__(THREADS) count_kernel(const int32_t* __restric
 }
 
 // One block: offs[e] = cumulative end of expert e; counts[b][e] becomes the first packed row
-// of block b's assignments to expert e.
+// of block b's assignments to expert e. G threads share an expert (G a power of two, at most
+// 32 and at most 1024 / E), each owning a contiguous run of blocks, so that the serial walk
+// over the histograms is nblk / G long instead of nblk.
 __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ counts, int32_t nblk,
                                                     int32_t E, int32_t* __restrict__ offs) {
+  __shared__ int32_t tot[GG_MAX_EXPERTS];  // per expert: total, then exclusive start
   __shared__ int32_t warp_sum[32];
-  const int e = threadIdx.x;
-  int32_t total = 0;
-  if (e < E)
-    for (int32_t b = 0; b < nblk; ++b) total += counts[(int64_t)b * E + e];
-  // block-wide inclusive scan of total over e
+  int lg = 5;
+  while (lg > 0 && (E << lg) > 1024) --lg;
+  const int G = 1 << lg;
+  const int e = threadIdx.x >> lg, s = threadIdx.x & (G - 1);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int32_t v = total;
+  const bool own = e < E;
+  const int32_t span = (nblk + G - 1) / G;
+  const int32_t b0 = min(s * span, nblk), b1 = min(b0 + span, nblk);
+  int32_t seg = 0;
+  if (own) {
+#pragma unroll 8
+    for (int32_t b = b0; b < b1; ++b) seg += counts[(int64_t)b * E + e];
+  }
+  // inclusive scan of the run sums over the G threads of the expert (a G-aligned lane group)
+  int32_t run_incl = seg;
+  for (int d = 1; d < G; d <<= 1) {
+    const int32_t o = __shfl_up_sync(0xffffffffu, run_incl, d);
+    if (s >= d) run_incl += o;
+  }
+  const int32_t total = __shfl_sync(0xffffffffu, run_incl, lane | (G - 1));
+  if (own && s == 0) tot[e] = total;
+  __syncthreads();
+  // block-wide exclusive scan of the totals over experts (thread x takes expert x)
+  const int32_t tx = (int)threadIdx.x < E ? tot[threadIdx.x] : 0;
+  int32_t v = tx;
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
     const int32_t o = __shfl_up_sync(0xffffffffu, v, d);
@@ -68,11 +89,14 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ counts
     warp_sum[lane] = w;
   }
   __syncthreads();
-  const int32_t incl = v + (warp > 0 ? warp_sum[warp - 1] : 0);
-  if (e < E) {
-    offs[e] = incl;
-    int32_t run = incl - total;
-    for (int32_t b = 0; b < nblk; ++b) {
+  if ((int)threadIdx.x < E) tot[threadIdx.x] = v + (warp > 0 ? warp_sum[warp - 1] : 0) - tx;
+  __syncthreads();
+  if (own) {
+    const int32_t start = tot[e];
+    if (s == 0) offs[e] = start + total;
+    int32_t run = start + run_incl - seg;
+#pragma unroll 8
+    for (int32_t b = b0; b < b1; ++b) {
       const int32_t c = counts[(int64_t)b * E + e];
       counts[(int64_t)b * E + e] = run;
       run += c;
@@ -109,15 +133,43 @@ __global__ void __launch_bounds__(THREADS) scatter_kernel(
   __syncthreads();
   const int32_t dest = valid ? whist[warp * E + e] + (int32_t)rank : -1;
   if (i < n) row_of[i] = dest;
-  // the warp copies its 32 rows, one after the other, each with all lanes
+  // Row copies. The lanes of one token are consecutive (i = t * k + slot), so the warp
+  // reads each token's row once, 512 bytes per lane step, and stores that piece to every
+  // destination of the token (reading the row once per slot re-read it from DRAM k times).
+  // Every loop below is warp-uniform: its bounds come from ballots and shuffles.
   const int64_t tok = i / k;
-  for (int j = 0; j < 32; ++j) {
-    const int32_t d = __shfl_sync(0xffffffffu, dest, j);
+  const int64_t tok_prev = __shfl_up_sync(0xffffffffu, tok, 1);
+  uint32_t leaders = __ballot_sync(0xffffffffu, i < n && (lane == 0 || tok != tok_prev));
+  const uint32_t has_dest = __ballot_sync(0xffffffffu, dest >= 0);
+  while (leaders != 0u) {
+    const int j = __ffs(leaders) - 1;
+    leaders &= leaders - 1u;
+    const int jend = leaders != 0u ? __ffs(leaders) - 1 : 32;
+    const uint32_t upto = jend == 32 ? 0xffffffffu : ((1u << jend) - 1u);
+    const uint32_t grp = upto & ~((1u << j) - 1u) & has_dest;  // lanes of this token
+    if (grp == 0u) continue;  // every slot of the token dropped
     const int64_t t = __shfl_sync(0xffffffffu, tok, j);
-    if (d < 0) continue;
     const uint4* src = X + t * row_vecs;
-    uint4* dst = A_packed + (int64_t)d * row_vecs;
-    for (int64_t v = lane; v < row_vecs; v += 32) dst[v] = src[v];
+    for (int64_t base = 0; base < row_vecs; base += 128) {
+      uint4 x[4] = {};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t v = base + lane + 32 * u;
+        if (v < row_vecs) x[u] = src[v];
+      }
+      uint32_t g = grp;
+      while (g != 0u) {
+        const int jj = __ffs(g) - 1;
+        g &= g - 1u;
+        const int32_t d = __shfl_sync(0xffffffffu, dest, jj);
+        uint4* dst = A_packed + (int64_t)d * row_vecs;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int64_t v = base + lane + 32 * u;
+          if (v < row_vecs) __stcs(dst + v, x[u]);  // written once, read by the next kernel
+        }
+      }
+    }
   }
 }
 

@@ -75,3 +75,23 @@ def test_watchdog_and_test_hook_setters(lib):
 def test_python_binding_has_no_fallback():
     src = open(os.path.join(ROOT, "moe_grouped_gemm_ragged_b200", "__init__.py")).read()
     assert "import oracle" not in src and "from oracle" not in src
+
+
+def test_host_step_checks_its_arguments_on_the_host(lib):
+    """gg_layer_step_host reads the offsets on the host (they are host data there) and rejects
+    decreasing or out-of-range offsets, bad sizes and null pointers before any CUDA call."""
+    f = lib.gg_layer_step_host
+    fake = ctypes.c_void_p(4096)
+
+    def args(offs, K=8, N=8, rows=16, first=fake):
+        o = ctypes.cast(offs, ctypes.c_void_p)
+        return [first, fake, fake, o, fake, fake, fake] + [fake] * 7 + [rows, K, N, 3, 0, None,
+                                                                        None]
+
+    assert f(*args((ctypes.c_int32 * 3)(8, 4, 12))) == 1    # decreasing
+    assert f(*args((ctypes.c_int32 * 3)(8, 12, 17))) == 1   # past the last row
+    assert f(*args((ctypes.c_int32 * 3)(-1, 4, 12))) == 1   # negative
+    good = (ctypes.c_int32 * 3)(4, 8, 12)
+    assert f(*args(good, K=12)) == 2                         # K not a multiple of 8
+    assert f(*args(good, first=None)) == 1                   # null pointer
+    assert f(*(args(good)[:14] + [16, 8, 8, 3, -1, None, None])) == 1  # negative chunk count
