@@ -469,6 +469,141 @@ def run_e2e(args, gg, r, m, dev, stream, ws, barrier):
             "expert_chunks": args.e2e_chunks or 8}
 
 
+def _median_call_ms(fn, stream, calls: int) -> float:
+    """Median of per-call CUDA-event times on ``stream`` after 3 warm-up calls."""
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(calls)]
+    for a, b in ev:
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return float(np.median([a.elapsed_time(b) for a, b in ev]))
+
+
+def _graph_call_us(fn, stream, calls: int) -> float:
+    """Per-call time of ``calls`` launches captured in one CUDA graph and replayed."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=torch.cuda.Stream()):
+        for _ in range(calls):
+            fn()
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    cur = torch.cuda.current_stream()
+    a.record(cur)
+    g.replay()
+    b.record(cur)
+    torch.cuda.synchronize()
+    del g
+    return a.elapsed_time(b) * 1e3 / calls
+
+
+def masked_bytes(m) -> int:
+    """Algorithmic bytes of the masked forward: active rows of A read once, W of the experts
+    with at least one active row read once, active output rows written once."""
+    act = np.clip(np.asarray(m.masked_m, np.int64), 0, m.mmax)
+    return int(act.sum() * (m.K + m.N) * 2 + (act > 0).sum() * m.K * m.N * 2)
+
+
+def run_table(args):
+    """Per-config, per-pass measurement of every parity config: GPU time (median of 20
+    calls; 200 for the tiny and masked shapes, which also report graph-replayed per-call
+    time), TFLOP/s and algorithmic GB/s, and the oracle's time on the host cores (in full
+    for tiny, masked and gate-up; on a row / K-row sample, extrapolated, for the others).
+    One JSON line per (config, pass)."""
+    import oracle
+    import workloads
+    import moe_grouped_gemm_ragged_b200 as gg
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (there is no CPU implementation)")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    peaks, _ = load_peaks()
+    threads = oracle.default_threads()
+
+    def emit(cfg, pas, flops, nbytes, ms, oracle_s, oracle_note, graph_us=None):
+        line = {"config": cfg, "pass": pas, "flops": flops, "algorithmic_bytes": nbytes,
+                "gpu_ms": ms, "tflops": flops / (ms * 1e-3) / 1e12,
+                "frac_of_burst_peak": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                "frac_of_spec_2250": flops / (ms * 1e-3) / 1e12 / 2250.0,
+                "gbs": nbytes / (ms * 1e-3) / 1e9,
+                "frac_of_hbm": nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                "graph_us_per_call": graph_us, "oracle_s": oracle_s,
+                "oracle_note": oracle_note, "oracle_threads": threads}
+        print(json.dumps(line), flush=True)
+
+    def ragged_bytes(r, pas):
+        T, K, N = r.T, r.K, r.N
+        live = int((np.asarray(r.sizes) > 0).sum())
+        w = live * K * N * 2
+        if pas == "forward":
+            return T * K * 2 + w + T * N * 2
+        if pas == "dgrad":
+            return T * N * 2 + w + T * K * 2
+        return T * (K + N) * 2 + r.E * K * N * 2
+
+    cases = [("tiny (8,16,32,40)", workloads.make_tiny((8, 16, 32, 40))),
+             ("tiny (8,8,32,40)", workloads.make_tiny((8, 8, 32, 40)))]
+    cases += [(n, None) for n in ("gateup", "downproj", "large", "large_unaligned")]
+    for cfg, r in cases:
+        if r is None:
+            r = workloads.make_ragged(cfg, tail=0, device=dev)
+        small = cfg.startswith("tiny")
+        A, W, dY = (t.to(dev) for t in (r.A, r.W, r.dY))
+        offs = torch.from_numpy(np.ascontiguousarray(r.offs)).to(dev)
+        out = torch.empty((r.rows_alloc, r.N), dtype=torch.bfloat16, device=dev)
+        dX = torch.empty((r.rows_alloc, r.K), dtype=torch.bfloat16, device=dev)
+        dW = torch.empty((r.E, r.K, r.N), dtype=torch.bfloat16, device=dev)
+        fns = {"forward": lambda: gg.forward(A, W, offs, out),
+               "dgrad": lambda: gg.dgrad(dY, W, offs, dX),
+               "wgrad": lambda: gg.wgrad(A, dY, offs, dW)}
+        hA, hW, hdY = oracle.as_u16(A), oracle.as_u16(W), oracle.as_u16(dY)
+        full = cfg.startswith("tiny") or cfg == "gateup"
+        rng = np.random.default_rng(0)
+        starts, ends, _ = oracle.group_bounds(r.offs, r.rows_alloc)
+        rows = None if full else np.concatenate(
+            [rng.integers(s, t, 16) for s, t in zip(starts, ends) if t > s]).astype(np.int64)
+        ks = None if full else np.sort(rng.choice(r.K, 8, replace=False)).astype(np.int64)
+        for pas, fn in fns.items():
+            ms = _median_call_ms(fn, stream, 200 if small else 20)
+            gus = _graph_call_us(fn, stream, 200) if small else None
+            t0 = time.perf_counter()
+            if pas == "forward":
+                oracle.forward(hA, hW, r.offs, rows=rows, threads=threads)
+            elif pas == "dgrad":
+                oracle.dgrad(hdY, hW, r.offs, rows=rows, threads=threads)
+            else:
+                oracle.wgrad(hA, hdY, r.offs, ks=ks, threads=threads)
+            osec = time.perf_counter() - t0
+            note = "full pass"
+            if not full:
+                frac = (len(rows) / max(1, r.T)) if pas != "wgrad" else len(ks) / r.K
+                osec /= frac
+                note = (f"extrapolated from {len(rows)} sampled rows" if pas != "wgrad"
+                        else f"extrapolated from {len(ks)} sampled K rows")
+            emit(cfg, pas, r.flops, ragged_bytes(r, pas), ms, osec, note, gus)
+        del A, W, dY, out, dX, dW
+        torch.cuda.empty_cache()
+
+    m = workloads.make_masked(device=dev)
+    mA, mW = m.A.to(dev), m.W.to(dev)
+    mm = torch.from_numpy(m.masked_m).to(dev)
+    mout = torch.empty((m.E, m.mmax, m.N), dtype=torch.bfloat16, device=dev)
+    fn = lambda: gg.masked_forward(mA, mW, mm, mout)  # noqa: E731
+    ms = _median_call_ms(fn, stream, 200)
+    gus = _graph_call_us(fn, stream, 200)
+    t0 = time.perf_counter()
+    oracle.masked_forward(oracle.as_u16(mA), oracle.as_u16(mW), m.masked_m, threads=threads)
+    osec = time.perf_counter() - t0
+    emit("masked", "forward", m.flops, masked_bytes(m), ms, osec, "full pass", gus)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -485,7 +620,11 @@ def main(argv=None):
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--variant", type=int, default=0, choices=[0, 1, 2],
                     help="launch shape of forward/dgrad: 0 automatic, 1 single CTA, 2 CTA pair")
+    ap.add_argument("--table", action="store_true",
+                    help="per-config, per-pass table of every parity config (JSON lines)")
     args = ap.parse_args(argv)
+    if args.table:
+        return run_table(args)
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

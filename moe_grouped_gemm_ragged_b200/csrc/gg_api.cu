@@ -159,7 +159,7 @@ template <Mode MODE, int BN, int STAGES, bool PAIR, bool F32 = false, int ACT = 
 gg_status launch(const CUtensorMap& a, const CUtensorMap& b, const gg::Params& p,
                  int64_t tiles_upper, const DeviceInfo& di, cudaStream_t stream) {
   auto kern = gg::grouped_gemm_kernel<MODE, BN, STAGES, PAIR, F32, ACT>;
-  using L = gg::Layout<BN, STAGES, PAIR>;
+  using L = gg::Layout<BN, STAGES, PAIR, gg::bk_of<MODE>()>;
   const size_t smem = L::bytes(p.E);
   int dev = 0;
   cudaError_t ce = cudaGetDevice(&dev);
@@ -264,6 +264,9 @@ constexpr int kBN = 256;
 constexpr int kStages = 4;      // single CTA: 48 KB per stage
 constexpr int kPairStages = 6;  // CTA pair: 32 KB per stage and CTA
 constexpr int kMaskedBN = 128;  // masked forward: 128 x 128 tiles, 32 KB per stage
+constexpr int kWgBK = gg::bk_of<Mode::Wgrad>();  // token rows per wgrad stage
+constexpr int kWgStages = kStages;
+constexpr int kWgPairStages = kPairStages;
 
 // CTA pairs halve the operand traffic per SM but quantise groups to 256-row tiles; they pay
 // off once the average group is long.
@@ -296,11 +299,11 @@ gg_status wgrad_impl(const void* A, const void* dY, const int32_t* offs, void* d
   const bool pair = g_force_variant.load() == 2;
   const uint32_t bcols = pair ? kBN / 2 : kBN;  // dY columns one CTA loads per stage
   CUtensorMap ma, mb;
-  if (a_chunked ? !map_2d_chunked(&ma, A, rows_alloc, K, 64, gg::BM / 64)
-                : !map_2d(&ma, A, rows_alloc, K, 64, 64))
+  if (a_chunked ? !map_2d_chunked(&ma, A, rows_alloc, K, kWgBK, gg::BM / 64)
+                : !map_2d(&ma, A, rows_alloc, K, 64, kWgBK))
     return GG_ERR_CUDA;
-  if (b_chunked ? !map_2d_chunked(&mb, dY, rows_alloc, N, 64, bcols / 64)
-                : !map_2d(&mb, dY, rows_alloc, N, 64, 64))
+  if (b_chunked ? !map_2d_chunked(&mb, dY, rows_alloc, N, kWgBK, bcols / 64)
+                : !map_2d(&mb, dY, rows_alloc, N, 64, kWgBK))
     return GG_ERR_CUDA;
   gg::Params p = base_params(offs, f32 ? nullptr : dW, dev_status, rows_alloc, E);
   p.out_cols = (int32_t)N;
@@ -314,12 +317,12 @@ gg_status wgrad_impl(const void* A, const void* dY, const int32_t* offs, void* d
   set_store_width(&p, dW, N);
   if (pair) {
     const int64_t tiles = (int64_t)E * cdiv(K, 2 * gg::BM) * cdiv(N, kBN);
-    if (f32) return launch<Mode::Wgrad, kBN, kPairStages, true, true>(ma, mb, p, tiles, di, stream);
-    return launch<Mode::Wgrad, kBN, kPairStages, true>(ma, mb, p, tiles, di, stream);
+    if (f32) return launch<Mode::Wgrad, kBN, kWgPairStages, true, true>(ma, mb, p, tiles, di, stream);
+    return launch<Mode::Wgrad, kBN, kWgPairStages, true>(ma, mb, p, tiles, di, stream);
   }
   const int64_t tiles = (int64_t)E * cdiv(K, gg::BM) * cdiv(N, kBN);
-  if (f32) return launch<Mode::Wgrad, kBN, kStages, false, true>(ma, mb, p, tiles, di, stream);
-  return launch<Mode::Wgrad, kBN, kStages, false>(ma, mb, p, tiles, di, stream);
+  if (f32) return launch<Mode::Wgrad, kBN, kWgStages, false, true>(ma, mb, p, tiles, di, stream);
+  return launch<Mode::Wgrad, kBN, kWgStages, false>(ma, mb, p, tiles, di, stream);
 }
 
 // Checks the epilogue description and stores it in p. act SiLU-and-mul needs N % 256 == 0

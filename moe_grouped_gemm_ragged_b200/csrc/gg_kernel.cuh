@@ -45,6 +45,11 @@ enum class Mode : int { Forward = 0, Dgrad = 1, Wgrad = 2, Masked = 3 };
 constexpr int BM = 128;         // tile rows (TMEM lanes)
 constexpr int BK = 64;          // reduction elements per stage (128 bytes of bf16)
 constexpr int UMMA_K = 16;      // reduction per tcgen05.mma for 16-bit inputs
+// Reduction elements per stage of each pass. All passes use BK: 32-row wgrad stages (twice
+// as many in the same shared memory) measured half the throughput on the large shape, each
+// stage taking about as long as a 64-row one.
+template <Mode MODE>
+__host__ __device__ constexpr int bk_of() { return BK; }
 constexpr int EPI_WARPS = 8;      // two per TMEM lane quadrant, each owning half the columns
 constexpr int FIX_WARP = 2 + EPI_WARPS;  // wgrad: zeroes the rows of a group's last stage
 constexpr int NUM_THREADS = 32 * (FIX_WARP + 1);
@@ -124,11 +129,13 @@ struct Params {
   int32_t zero_tail;
 };
 
-template <int BN, int STAGES, bool PAIR>
+template <int BN, int STAGES, bool PAIR, int BKL = BK>
 struct Layout {
   static constexpr int B_COLS = PAIR ? BN / 2 : BN;  // columns of B this CTA loads
-  static constexpr uint32_t A_BYTES = BM * BK * 2;
-  static constexpr uint32_t B_BYTES = B_COLS * BK * 2;
+  static constexpr uint32_t A_BYTES = BM * BKL * 2;
+  static constexpr uint32_t B_BYTES = B_COLS * BKL * 2;
+  // an MN-major operand holds one BKL-row x 128-byte block per 64-wide chunk
+  static constexpr uint32_t CHUNK_BYTES = BKL * 128;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr uint32_t OFF_A = 0;
   static constexpr uint32_t OFF_B = STAGES * A_BYTES;
@@ -332,7 +339,7 @@ __device__ __forceinline__ Tile decode_tile(int32_t t, const Params& p, const Sh
     tl.n0 = nt * BN;
     tl.tok0 = sh.gstart[e];
     tl.tok_len = sh.gend[e] - sh.gstart[e];
-    tl.kblocks = (tl.tok_len + BK - 1) / BK;
+    tl.kblocks = (tl.tok_len + bk_of<MODE>() - 1) / bk_of<MODE>();
     tl.row0 = (int64_t)e * p.wg_K + tl.k0;
     tl.row_end = (int64_t)e * p.wg_K + p.wg_K;
     tl.a_row0 = 0;
@@ -352,7 +359,7 @@ __device__ __forceinline__ Tile decode_tile(int32_t t, const Params& p, const Sh
     tl.row0 = tl.a_row0;
     tl.row_end = sh.gend[e];
     tl.n0 = nt * BN;
-    tl.kblocks = e < p.E ? (p.red_len + BK - 1) / BK : 0;
+    tl.kblocks = e < p.E ? (p.red_len + bk_of<MODE>() - 1) / bk_of<MODE>() : 0;
     tl.k0 = 0;
     tl.tok0 = 0;
     tl.tok_len = 0;
@@ -366,7 +373,8 @@ template <Mode MODE, int BN, int STAGES, bool PAIR, bool F32 = false, int ACT = 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap mapA,
                         const __grid_constant__ CUtensorMap mapB, const Params p) {
-  using L = Layout<BN, STAGES, PAIR>;
+  constexpr int BKM = bk_of<MODE>();  // reduction elements per stage
+  using L = Layout<BN, STAGES, PAIR, BKM>;
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN must be 64, 128, 192 or 256");
   static_assert(!PAIR || BN % 128 == 0, "a CTA pair splits BN into two multiples of 64");
   static_assert(L::TMEM_COLS == 128 || L::TMEM_COLS == 256 || L::TMEM_COLS == 512,
@@ -473,16 +481,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint8_t* sA = smem + L::OFF_A + stage * L::A_BYTES;
         uint8_t* sB = smem + L::OFF_B + stage * L::B_BYTES;
         uint64_t* fb = &sh.full[stage];
-        int32_t rem = BK;  // wgrad: rows of the group in this stage
-        if constexpr (MODE == Mode::Wgrad) rem = tl.tok_len - kb * BK;
-        const bool tail = MODE == Mode::Wgrad && rem < BK;
+        int32_t rem = BKM;  // wgrad: rows of the group in this stage
+        if constexpr (MODE == Mode::Wgrad) rem = tl.tok_len - kb * BKM;
+        const bool tail = MODE == Mode::Wgrad && rem < BKM;
         if (lane == 0) {
           armed &= ~(1u << stage);
           armed_l &= ~(1u << stage);
           if (skip_first) {
             skip_first = false;  // watchdog test: this stage is never armed
           } else if constexpr (PAIR && MODE == Mode::Wgrad) {
-            const int32_t r = tl.tok0 + kb * BK;
+            const int32_t r = tl.tok0 + kb * BKM;
             const int32_t ka = tl.k0 + row_off;  // this CTA's 128 columns of A (K)
             const int32_t nb = tl.n0 + col_off;  // this CTA's columns of dY (N)
             if (tail) {
@@ -495,13 +503,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 ptx::tma_load_3d(sA, &mapA, lb, 0, r, ka / 64, pol_wg);
               } else {
                 for (int j = 0; j < 2; ++j)
-                  ptx::tma_load_2d(sA + j * 8192, &mapA, lb, ka + j * 64, r, pol_wg);
+                  ptx::tma_load_2d(sA + j * L::CHUNK_BYTES, &mapA, lb, ka + j * 64, r, pol_wg);
               }
               if (p.b_chunked) {
                 ptx::tma_load_3d(sB, &mapB, lb, 0, r, nb / 64, pol_wg);
               } else {
                 for (int j = 0; j < L::B_COLS / 64; ++j)
-                  ptx::tma_load_2d(sB + j * 8192, &mapB, lb, nb + j * 64, r, pol_wg);
+                  ptx::tma_load_2d(sB + j * L::CHUNK_BYTES, &mapB, lb, nb + j * 64, r, pol_wg);
               }
             } else {
               const uint32_t fb_leader = ptx::mapa(ptx::smem_u32(fb), 0);
@@ -510,13 +518,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 ptx::tma_load_3d_pair(sA, &mapA, fb_leader, 0, r, ka / 64, pol_wg);
               } else {
                 for (int j = 0; j < 2; ++j)
-                  ptx::tma_load_2d_pair(sA + j * 8192, &mapA, fb_leader, ka + j * 64, r, pol_wg);
+                  ptx::tma_load_2d_pair(sA + j * L::CHUNK_BYTES, &mapA, fb_leader, ka + j * 64, r, pol_wg);
               }
               if (p.b_chunked) {
                 ptx::tma_load_3d_pair(sB, &mapB, fb_leader, 0, r, nb / 64, pol_wg);
               } else {
                 for (int j = 0; j < L::B_COLS / 64; ++j)
-                  ptx::tma_load_2d_pair(sB + j * 8192, &mapB, fb_leader, nb + j * 64, r, pol_wg);
+                  ptx::tma_load_2d_pair(sB + j * L::CHUNK_BYTES, &mapB, fb_leader, nb + j * 64, r, pol_wg);
               }
               if (leader) {
                 armed |= 1u << stage;
@@ -527,17 +535,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             // the leader's full barrier counts the bytes of both CTAs
             const uint32_t fb_leader = ptx::mapa(ptx::smem_u32(fb), 0);
             if (leader) ptx::mbar_arrive_expect_tx(fb, 2 * L::STAGE_BYTES);
-            ptx::tma_load_2d_pair(sA, &mapA, fb_leader, kb * BK, tl.a_row0 + row_off, pol_tok);
+            ptx::tma_load_2d_pair(sA, &mapA, fb_leader, kb * BKM, tl.a_row0 + row_off, pol_tok);
             if constexpr (MODE == Mode::Dgrad) {
-              ptx::tma_load_3d_pair(sB, &mapB, fb_leader, kb * BK, tl.n0 + col_off, tl.e, pol_w);
+              ptx::tma_load_3d_pair(sB, &mapB, fb_leader, kb * BKM, tl.n0 + col_off, tl.e, pol_w);
             } else if (p.b_chunked) {
-              ptx::tma_load_4d_pair(sB, &mapB, fb_leader, 0, kb * BK, (tl.n0 + col_off) / 64,
+              ptx::tma_load_4d_pair(sB, &mapB, fb_leader, 0, kb * BKM, (tl.n0 + col_off) / 64,
                                     tl.e, pol_w);
             } else {
 #pragma unroll
               for (int j = 0; j < L::B_COLS / 64; ++j)
-                ptx::tma_load_3d_pair(sB + j * 8192, &mapB, fb_leader, tl.n0 + col_off + j * 64,
-                                      kb * BK, tl.e, pol_w);
+                ptx::tma_load_3d_pair(sB + j * L::CHUNK_BYTES, &mapB, fb_leader, tl.n0 + col_off + j * 64,
+                                      kb * BKM, tl.e, pol_w);
             }
             if (leader) {
               armed |= 1u << stage;
@@ -554,38 +562,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               const int32_t nbox = (int32_t)((valid + 31) / 32);
               ptx::mbar_arrive_expect_tx(lb, (uint32_t)nbox * 32u * 128u + L::B_BYTES);
               for (int32_t b = 0; b < nbox; ++b)
-                ptx::tma_load_2d(sA + b * 4096, &mapA, lb, kb * BK, tl.a_row0 + b * 32, pol_tok);
+                ptx::tma_load_2d(sA + b * 4096, &mapA, lb, kb * BKM, tl.a_row0 + b * 32, pol_tok);
             } else {
               ptx::mbar_arrive_expect_tx(lb, L::STAGE_BYTES);
             }
             if constexpr (MODE == Mode::Forward || MODE == Mode::Masked) {
               if constexpr (MODE == Mode::Forward)
-                ptx::tma_load_2d(sA, &mapA, lb, kb * BK, tl.a_row0, pol_tok);
+                ptx::tma_load_2d(sA, &mapA, lb, kb * BKM, tl.a_row0, pol_tok);
               if (p.b_chunked) {
-                ptx::tma_load_4d(sB, &mapB, lb, 0, kb * BK, tl.n0 / 64, tl.e, pol_w);
+                ptx::tma_load_4d(sB, &mapB, lb, 0, kb * BKM, tl.n0 / 64, tl.e, pol_w);
               } else {
 #pragma unroll
                 for (int j = 0; j < BN / 64; ++j)
-                  ptx::tma_load_3d(sB + j * 8192, &mapB, lb, tl.n0 + j * 64, kb * BK, tl.e, pol_w);
+                  ptx::tma_load_3d(sB + j * L::CHUNK_BYTES, &mapB, lb, tl.n0 + j * 64, kb * BKM, tl.e, pol_w);
               }
             } else if constexpr (MODE == Mode::Dgrad) {
-              ptx::tma_load_2d(sA, &mapA, lb, kb * BK, tl.a_row0, pol_tok);
-              ptx::tma_load_3d(sB, &mapB, lb, kb * BK, tl.n0, tl.e, pol_w);
+              ptx::tma_load_2d(sA, &mapA, lb, kb * BKM, tl.a_row0, pol_tok);
+              ptx::tma_load_3d(sB, &mapB, lb, kb * BKM, tl.n0, tl.e, pol_w);
             } else {  // Wgrad
-              const int32_t r = tl.tok0 + kb * BK;
+              const int32_t r = tl.tok0 + kb * BKM;
               if (p.a_chunked) {
                 ptx::tma_load_3d(sA, &mapA, lb, 0, r, tl.k0 / 64, pol_wg);
               } else {
 #pragma unroll
                 for (int j = 0; j < 2; ++j)
-                  ptx::tma_load_2d(sA + j * 8192, &mapA, lb, tl.k0 + j * 64, r, pol_wg);
+                  ptx::tma_load_2d(sA + j * L::CHUNK_BYTES, &mapA, lb, tl.k0 + j * 64, r, pol_wg);
               }
               if (p.b_chunked) {
                 ptx::tma_load_3d(sB, &mapB, lb, 0, r, tl.n0 / 64, pol_wg);
               } else {
 #pragma unroll
                 for (int j = 0; j < BN / 64; ++j)
-                  ptx::tma_load_2d(sB + j * 8192, &mapB, lb, tl.n0 + j * 64, r, pol_wg);
+                  ptx::tma_load_2d(sB + j * L::CHUNK_BYTES, &mapB, lb, tl.n0 + j * 64, r, pol_wg);
               }
             }
             if (!tail) {
@@ -620,7 +628,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // descriptor deltas per 16-element reduction step (address field is in 16-byte units)
       constexpr uint64_t A_STEP = A_MN ? (2048u >> 4) : (32u >> 4);
       constexpr uint64_t B_STEP = B_MN ? (2048u >> 4) : (32u >> 4);
-      const uint32_t a_lbo = A_MN ? 8192u : 16u, b_lbo = B_MN ? 8192u : 16u;
+      const uint32_t a_lbo = A_MN ? L::CHUNK_BYTES : 16u, b_lbo = B_MN ? L::CHUNK_BYTES : 16u;
       uint32_t stage = 0, phase = 0, acc_iter = 0;
       uint32_t fixed_par = 0;  // per stage: next phase of fixed[] (pair wgrad)
       bool ok = true;
@@ -641,10 +649,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #if GG_FENCE_PER_STAGE
           ptx::tc_fence_after();
 #endif
-          int nsub = BK / UMMA_K;
+          int nsub = BKM / UMMA_K;
           if constexpr (MODE == Mode::Wgrad) {
-            const int32_t rem = tl.tok_len - kb * BK;
-            if (rem < BK) {
+            const int32_t rem = tl.tok_len - kb * BKM;
+            if (rem < BKM) {
               nsub = (rem + UMMA_K - 1) / UMMA_K;
               if constexpr (PAIR_WGRAD) {
                 // the follower's half of this stage is fixed up on its own schedule
@@ -659,7 +667,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint64_t bdesc = ptx::smem_desc_sw128(
               ptx::smem_u32(smem + L::OFF_B + stage * L::B_BYTES), b_lbo, 1024);
 #pragma unroll
-          for (int k = 0; k < BK / UMMA_K; ++k) {
+          for (int k = 0; k < BKM / UMMA_K; ++k) {
             if (k < nsub) {
               const uint32_t acc = (kq > 0 || k > 0) ? 1u : 0u;  // the first stage overwrites
               if constexpr (PAIR)
@@ -911,8 +919,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       for (int32_t kq = 0; kq < tl.kblocks; ++kq) {
         const int32_t kb = rev ? tl.kblocks - 1 - kq : kq;
-        const int32_t rem = tl.tok_len - kb * BK;
-        if (rem < BK) {
+        const int32_t rem = tl.tok_len - kb * BKM;
+        if (rem < BKM) {
           const uint32_t lp = (landed_par >> stage) & 1u;
           landed_par ^= 1u << stage;
           if (!warp_wait(&sh.landed[stage], lp, sh, p, false)) { ok = false; break; }
@@ -925,10 +933,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const int line = i >> 3, part = i & 7;
             uint8_t* dst;
             if (line < lines_a) {
-              dst = sA + (line / zrows) * 8192 + (rem + line % zrows) * 128 + part * 16;
+              dst = sA + (line / zrows) * L::CHUNK_BYTES + (rem + line % zrows) * 128 + part * 16;
             } else {
               const int l2 = line - lines_a;
-              dst = sB + (l2 / zrows) * 8192 + (rem + l2 % zrows) * 128 + part * 16;
+              dst = sB + (l2 / zrows) * L::CHUNK_BYTES + (rem + l2 % zrows) * 128 + part * 16;
             }
             *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
           }
