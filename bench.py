@@ -39,12 +39,12 @@ UNIT = "TFLOP/s"
 #   --clock-control none -k regex:grouped_gemm -s 12 -c 4 python bench.py --steps 1 --warmup 3
 #   --no-e2e --no-cpu   (see profiles/grouped_gemm_large_launch_list.md)
 NCU_TRAFFIC = {
-    ("forward", "large"): 12.376e9,
-    ("dgrad", "large"): 11.844e9,
-    ("wgrad", "large"): 14.618e9,
+    ("forward", "large"): 19.379e9,
+    ("dgrad", "large"): 16.831e9,
+    ("wgrad", "large"): 14.671e9,
     ("masked", "large"): 0.023e9,
 }
-NCU_TRAFFIC_SRC_HASH = "cb440b395283ee9a"
+NCU_TRAFFIC_SRC_HASH = "28188f2a8090e536"
 
 
 GEMM_SOURCES = ("gg_kernel.cuh", "ptx.cuh", "gg_api.cu")  # the grouped GEMM kernels + launch
@@ -466,7 +466,7 @@ def run_e2e(args, gg, r, m, dev, stream, ws, barrier):
     return {"value": ws * flops / (ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms,
             "steps": steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "api": "gg_layer_step_host + gg_masked_forward",
-            "expert_chunks": args.e2e_chunks or 8}
+            "expert_chunks": args.e2e_chunks or 16}
 
 
 def _median_call_ms(fn, stream, calls: int) -> float:

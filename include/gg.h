@@ -16,8 +16,8 @@
  * any size; no alignment is asked of the sizes (TransformerEngine PR 3224 names an
  * alignment contract on m_splits that this library does not have).
  *
- * Offsets and masked_m are read only on the device ("expert counts remain on the GPU",
- * TransformerEngine PR 3542, "Changes"). No call synchronises with the host, allocates
+ * Offsets and masked_m are read only on the device (TransformerEngine PR 3542, "Changes":
+ * the per-expert row counts stay in GPU memory). No call synchronises with the host, allocates
  * memory, pads A or clears an output (TileOPs issue 1566, "Summary": the per-call zero
  * fill and pad cost ~2.8 ms on a ~20 ms GEMM). Every call is ordered on the caller's
  * stream and may be captured in a CUDA graph; the offsets may change between replays.
@@ -26,8 +26,8 @@
  * (last index contiguous) and 16-byte aligned. W is one packed [E,K,N] buffer (the single
  * grouped weight of TransformerEngine PR 3224). K and N must be multiples of 8.
  *
- * Untouched regions ("caller-owned output buffers and unused capacity are preserved",
- * TransformerEngine PR 3542, "Changes"):
+ * Untouched regions (TransformerEngine PR 3542, "Changes": outputs live in buffers the caller
+ * owns, and their rows beyond the used capacity keep their contents):
  *   - out/dX rows at or past the last (effective) offset are never written, and A/dY rows
  *     there are never read into any result;
  *   - masked rows r >= masked_m[e] of out are never written; A rows there never reach a
@@ -167,8 +167,8 @@ GG_API gg_status gg_masked_forward(const void* A, const void* W, const int32_t* 
  *                        of 256 columns (N % 256 == 0, else GG_ERR_UNSUPPORTED):
  *                        out[r, 128 b + i] = silu(h[r, 256 b + i]) * h[r, 256 b + 128 + i],
  *                        silu(x) = x / (1 + e^-x)                 (out has N / 2 columns)
- * Passages: TransformerEngine PR 3542 review ("Expand per-group bias across result capacity",
- * "Per-token bias scale", scaling limited to the logical rows); sglang PR 32385, "Cause"
+ * Passages: TransformerEngine PR 3542 review (a bias per group, a bias scale per token, the
+ * scaling limited to the logical rows and not the capacity); sglang PR 32385, "Cause"
  * (SiLU-and-mul between the gate-up and the down GEMM, written only for active rows). */
 #define GG_ACT_NONE 0
 #define GG_ACT_SILU_MUL 1
@@ -178,7 +178,8 @@ GG_API gg_status gg_masked_forward(const void* A, const void* W, const int32_t* 
  *                      of being left untouched
  *   GG_FLAG_W_NK       W (and dW) stored [E, N, K]: each expert's weight out-major, the way
  *                      TransformerEngine's GroupedLinear keeps it (TransformerEngine PR 3542,
- *                      "Adds TN, NN, and NT dispatch"); forward computes A . W[e]^T */
+ *                      "Changes": dispatch of the transposed operand layouts); forward
+ *                      computes A . W[e]^T */
 #define GG_FLAG_ZERO_TAIL 0x1
 #define GG_FLAG_W_NK 0x2
 typedef struct gg_epilogue {
@@ -256,7 +257,7 @@ GG_API gg_status gg_route_noalloc(const int32_t* topk_ids, int64_t T_tok, int32_
  *     not written.
  *   device staging, caller-owned, the same shapes: A_d, W_d, dY_d, out_d, dX_d, dW_d, and
  *     offs_d int32 [E], which ends up holding chunk-relative offsets.
- *   chunks: number of expert chunks (0: 8; at most E and 32).
+ *   chunks: number of expert chunks (0: 16; at most E and 32).
  * The offsets are host data here and are checked on the host: non-decreasing within
  * [0, rows], else GG_ERR_INVALID_ARG and nothing is enqueued. The call returns once all work
  * is enqueued; `stream` is ordered after the last copy back, so the host results are valid

@@ -14,7 +14,7 @@ namespace ggh {
 
 constexpr int kMaxChunks = 32;
 constexpr int kMaxDevices = 64;
-constexpr int kDefaultChunks = 8;
+constexpr int kDefaultChunks = 16;
 
 // Per device: the two copy streams and the events that order the three streams. They are
 // created on first use and kept; one process-wide lock serialises the enqueueing, and an
