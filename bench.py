@@ -618,8 +618,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-extras", action="store_true")
-    ap.add_argument("--variant", type=int, default=0, choices=[0, 1, 2],
-                    help="launch shape of forward/dgrad: 0 automatic, 1 single CTA, 2 CTA pair")
+    ap.add_argument("--variant", type=int, default=0, choices=[0, 1, 2, 3],
+                    help="launch shapes: 0 automatic, 1 single CTA, 2 CTA pair, 3 CTA pair with 256 x 512 wgrad tiles")
     ap.add_argument("--table", action="store_true",
                     help="per-config, per-pass table of every parity config (JSON lines)")
     args = ap.parse_args(argv)

@@ -32,7 +32,8 @@ gg_status cuda_fail(const char* where, cudaError_t e) {
   return GG_ERR_CUDA;
 }
 std::atomic<int> g_skip_first_load{0};
-std::atomic<int> g_force_variant{0};  // test hook: 0 automatic, 1 single CTA, 2 CTA pair
+// test hook: 0 automatic, 1 single CTA, 2 CTA pair, 3 CTA pair with 512-column wgrad tiles
+std::atomic<int> g_force_variant{0};
 
 static_assert(gg::DEV_BAD_OFFSETS == GG_DEV_BAD_OFFSETS, "status bit mismatch");
 static_assert(gg::DEV_BAD_MASKED_M == GG_DEV_BAD_MASKED_M, "status bit mismatch");
@@ -267,14 +268,45 @@ constexpr int kMaskedBN = 128;  // masked forward: 128 x 128 tiles, 32 KB per st
 constexpr int kWgBK = gg::bk_of<Mode::Wgrad>();  // token rows per wgrad stage
 constexpr int kWgStages = kStages;
 constexpr int kWgPairStages = kPairStages;
+// Wide CTA-pair tiles: 256 x 512 with one accumulator (all 512 TMEM columns), 48 KB per
+// stage and CTA. Per flop they move a quarter less operand data into shared memory than
+// 256 x 256 pair tiles and, in wgrad, cover twice as much of dW per wave.
+constexpr int kWideBN = 512;
+constexpr int kWideStages = 4;
 
 // CTA pairs halve the operand traffic per SM but quantise groups to 256-row tiles; they pay
 // off once the average group is long.
 bool use_pair(int64_t rows, int32_t E) {
   const int v = g_force_variant.load();
   if (v == 1) return false;
-  if (v == 2) return true;
+  if (v == 2 || v == 3) return true;
   return rows >= 512 * (int64_t)E;
+}
+
+// Forward and dgrad on 256 x 512 CTA-pair tiles where CTA pairs are used and the reduction
+// is long: the tile's epilogue no longer overlaps the next mainloop, which a long reduction
+// amortises (large shape, reduction 6144 / 4096: forward 1279 vs 1205 TFLOP/s, dgrad 1219 vs
+// 1188 in alternating runs; down-proj forward, reduction 2048: 1158 vs 1221).
+bool use_wide(int64_t rows, int32_t E, int64_t red_len) {
+  const int v = g_force_variant.load();
+  if (v == 1 || v == 2) return false;
+  if (v == 3) return true;
+  return rows >= 512 * (int64_t)E && red_len >= 4096;
+}
+
+// Wgrad launch shape: 0 single CTAs, 1 CTA pairs, 2 wide CTA pairs. A wgrad tile is as long
+// as its expert, so the shapes trade per-stage efficiency against balance: wide pairs on
+// long groups (large shape 1363 TFLOP/s vs 1181 single, 1134 pair; down-proj 1333 vs 1144,
+// 1205), plain pairs on the Zipf gate-up shape (average 512 rows: 776 vs 737 single, 731
+// wide), single CTAs below.
+int wgrad_shape(int64_t rows, int32_t E) {
+  const int v = g_force_variant.load();
+  if (v == 1) return 0;
+  if (v == 2) return 1;
+  if (v == 3) return 2;
+  if (rows >= 1024 * (int64_t)E) return 2;
+  if (rows >= 256 * (int64_t)E) return 1;
+  return 0;
 }
 
 gg_status wgrad_impl(const void* A, const void* dY, const int32_t* offs, void* dW, bool f32,
@@ -294,10 +326,13 @@ gg_status wgrad_impl(const void* A, const void* dY, const int32_t* offs, void* d
     dY = dW;
   }
   const bool a_chunked = (K % 64) == 0, b_chunked = (N % 64) == 0;
-  // wgrad stays on single CTAs unless forced: measured faster on long groups (large shape
-  // 1159 vs 909 TFLOP/s) and equal on short ones
-  const bool pair = g_force_variant.load() == 2;
-  const uint32_t bcols = pair ? kBN / 2 : kBN;  // dY columns one CTA loads per stage
+  // Single CTAs with 128 x 256 tiles, CTA pairs with 256 x 256 tiles, or CTA pairs with
+  // 256 x 512 tiles and one accumulator: the tiles in flight then cover twice as much of an
+  // expert's dW, so each operand row streams from HBM half as often.
+  const int shape = wgrad_shape(rows_alloc, E);
+  const bool wide = shape == 2;
+  const bool pair = shape >= 1;
+  const uint32_t bcols = wide ? kWideBN / 2 : pair ? kBN / 2 : kBN;  // dY columns per CTA
   CUtensorMap ma, mb;
   if (a_chunked ? !map_2d_chunked(&ma, A, rows_alloc, K, kWgBK, gg::BM / 64)
                 : !map_2d(&ma, A, rows_alloc, K, 64, kWgBK))
@@ -315,6 +350,12 @@ gg_status wgrad_impl(const void* A, const void* dY, const int32_t* offs, void* d
   p.alpha = alpha;
   p.beta = beta;
   set_store_width(&p, dW, N);
+  if (wide) {
+    const int64_t tiles = (int64_t)E * cdiv(K, 2 * gg::BM) * cdiv(N, kWideBN);
+    if (f32)
+      return launch<Mode::Wgrad, kWideBN, kWideStages, true, true>(ma, mb, p, tiles, di, stream);
+    return launch<Mode::Wgrad, kWideBN, kWideStages, true>(ma, mb, p, tiles, di, stream);
+  }
   if (pair) {
     const int64_t tiles = (int64_t)E * cdiv(K, 2 * gg::BM) * cdiv(N, kBN);
     if (f32) return launch<Mode::Wgrad, kBN, kWgPairStages, true, true>(ma, mb, p, tiles, di, stream);
@@ -357,8 +398,9 @@ gg_status forward_impl(const void* A, const void* W, const int32_t* offs, void* 
   const bool silu = epi != nullptr && epi->act == GG_ACT_SILU_MUL;
   const bool wnk = (flags & GG_FLAG_W_NK) != 0;
   const bool pair = use_pair(rows_alloc, E);
+  const bool wide = pair && !silu && use_wide(rows_alloc, E, K);
   const bool chunked = (N % 64) == 0;
-  const uint32_t bcols = pair ? kBN / 2 : kBN;
+  const uint32_t bcols = wide ? kWideBN / 2 : pair ? kBN / 2 : kBN;
   CUtensorMap ma, mb;
   if (!map_2d(&ma, A, rows_alloc, K, 64, gg::BM)) return GG_ERR_CUDA;
   if (wnk) {
@@ -377,7 +419,12 @@ gg_status forward_impl(const void* A, const void* W, const int32_t* offs, void* 
   p.out_cols = (int32_t)out_cols;
   p.prod_cols = (int32_t)N;
   set_store_width(&p, out, out_cols);
-  const int64_t tiles = (cdiv(rows_alloc, (pair ? 2 : 1) * gg::BM) + E + 1) * cdiv(N, kBN);
+  const int64_t tiles =
+      (cdiv(rows_alloc, (pair ? 2 : 1) * gg::BM) + E + 1) * cdiv(N, wide ? kWideBN : kBN);
+  if (wide) {
+    if (wnk) return launch<Mode::Dgrad, kWideBN, kWideStages, true>(ma, mb, p, tiles, di, stream);
+    return launch<Mode::Forward, kWideBN, kWideStages, true>(ma, mb, p, tiles, di, stream);
+  }
   if (wnk) {
     if (pair) {
       if (silu) return launch<Mode::Dgrad, kBN, kPairStages, true, false, 1>(ma, mb, p, tiles, di, stream);
@@ -409,7 +456,8 @@ gg_status dgrad_impl(const void* dY, const void* W, const int32_t* offs, void* d
   if (!aligned16(dY) || !aligned16(W) || !aligned16(dX)) return GG_ERR_UNSUPPORTED;
   const bool wnk = (flags & GG_FLAG_W_NK) != 0;
   const bool pair = use_pair(rows_alloc, E);
-  const uint32_t bcols = pair ? kBN / 2 : kBN;
+  const bool wide = pair && use_wide(rows_alloc, E, N);
+  const uint32_t bcols = wide ? kWideBN / 2 : pair ? kBN / 2 : kBN;
   const bool chunked = (K % 64) == 0;
   CUtensorMap ma, mb;
   if (!map_2d(&ma, dY, rows_alloc, N, 64, gg::BM)) return GG_ERR_CUDA;
@@ -428,7 +476,12 @@ gg_status dgrad_impl(const void* dY, const void* W, const int32_t* offs, void* d
   p.b_chunked = (wnk && chunked) ? 1 : 0;
   p.zero_tail = (flags & GG_FLAG_ZERO_TAIL) ? 1 : 0;
   set_store_width(&p, dX, K);
-  const int64_t tiles = (cdiv(rows_alloc, (pair ? 2 : 1) * gg::BM) + E + 1) * cdiv(K, kBN);
+  const int64_t tiles =
+      (cdiv(rows_alloc, (pair ? 2 : 1) * gg::BM) + E + 1) * cdiv(K, wide ? kWideBN : kBN);
+  if (wide) {
+    if (wnk) return launch<Mode::Forward, kWideBN, kWideStages, true>(ma, mb, p, tiles, di, stream);
+    return launch<Mode::Dgrad, kWideBN, kWideStages, true>(ma, mb, p, tiles, di, stream);
+  }
   if (wnk) {
     if (pair) return launch<Mode::Forward, kBN, kPairStages, true>(ma, mb, p, tiles, di, stream);
     return launch<Mode::Forward, kBN, kStages, false>(ma, mb, p, tiles, di, stream);
@@ -558,7 +611,7 @@ uint64_t gg_set_watchdog_ns(uint64_t ns) {
 int gg_testing_skip_first_load(int enable) { return g_skip_first_load.exchange(enable ? 1 : 0); }
 
 int gg_testing_force_variant(int variant) {
-  return g_force_variant.exchange(variant == 1 || variant == 2 ? variant : 0);
+  return g_force_variant.exchange(variant >= 1 && variant <= 3 ? variant : 0);
 }
 
 int gg_version(void) { return 100; }

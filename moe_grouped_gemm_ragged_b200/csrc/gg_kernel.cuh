@@ -144,7 +144,11 @@ struct Layout {
   static constexpr uint32_t NUM_BARS = 4 * STAGES + 5;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr uint32_t OFF_TAB = OFF_MISC + 16;
-  static constexpr uint32_t TMEM_COLS = 2 * BN;
+  // fp32 accumulators in tensor memory: two of BN columns (the epilogue drains one while the
+  // next tile fills the other), or one when a tile is wider than 256 columns (512 columns,
+  // all of an SM's tensor memory)
+  static constexpr uint32_t ACC_BUFS = BN > 256 ? 1 : 2;
+  static constexpr uint32_t TMEM_COLS = ACC_BUFS * BN;
   // gstart[E+1], gend[E+1], prefix[E+2], order[E] (int32); group E is the zero tail
   static __host__ __device__ constexpr uint32_t bytes(int E) {
     return OFF_TAB + 4u * (4u * ((uint32_t)E + 1u) + 1u) + 1024u /* alignment slack */;
@@ -387,7 +391,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         const __grid_constant__ CUtensorMap mapB, const Params p) {
   constexpr int BKM = bk_of<MODE>();  // reduction elements per stage
   using L = Layout<BN, STAGES, PAIR, BKM>;
-  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN must be 64, 128, 192 or 256");
+  static_assert(BN % 64 == 0 && BN >= 64 && (BN <= 256 || (BN == 512 && PAIR)),
+                "BN must be 64, 128, 192 or 256, or 512 for a CTA pair");
   static_assert(!PAIR || BN % 128 == 0, "a CTA pair splits BN into two multiples of 64");
   static_assert(L::TMEM_COLS == 128 || L::TMEM_COLS == 256 || L::TMEM_COLS == 512,
                 "TMEM allocation must be a power of two");
@@ -395,7 +400,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // A operand MN-major only in Wgrad; B operand K-major only in Dgrad.
   constexpr uint32_t A_MN = (MODE == Mode::Wgrad) ? 1u : 0u;
   constexpr uint32_t B_MN = (MODE == Mode::Dgrad) ? 0u : 1u;
-  constexpr uint32_t IDESC = ptx::idesc_bf16_f32(TM, BN, A_MN, B_MN);
+  // One MMA covers at most 256 columns; a 512-column pair tile issues two per reduction step,
+  // each taking 128 of the 256 B columns that each CTA holds (TMEM columns [256h, 256h+256)
+  // of MMA h: the first 128 from the leader's B, the next 128 from the follower's).
+  constexpr int MMA_N = BN > 256 ? 256 : BN;
+  constexpr int NSPLIT = BN / MMA_N;
+  constexpr uint32_t IDESC = ptx::idesc_bf16_f32(TM, MMA_N, A_MN, B_MN);
   constexpr uint32_t EPI_ARRIVALS = (PAIR ? 2u : 1u) * EPI_WARPS;  // one per epilogue warp
   // In a pair's wgrad, the follower signals its fixed-up half of a group's last stage on the
   // leader's fixed[] barrier (a stage with whole rows only completes by its byte count).
@@ -650,8 +660,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const Tile tl = decode_tile<MODE, BN, TM>(t, p, sh);
         if (tl.kblocks == 0) continue;  // Wgrad of an empty expert: the epilogue writes zeros
         const bool rev = GG_SERPENTINE && (it & 1);
-        const uint32_t a = acc_iter & 1u;
-        if (!wait_bounded(&sh.tempty[a], ((acc_iter >> 1) & 1u) ^ 1u, sh, p, true, PAIR)) {
+        const uint32_t a = acc_iter % L::ACC_BUFS;
+        if (!wait_bounded(&sh.tempty[a], ((acc_iter / L::ACC_BUFS) & 1u) ^ 1u, sh, p, true,
+                          PAIR)) {
           ok = false;
           break;
         }
@@ -684,10 +695,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int k = 0; k < BKM / UMMA_K; ++k) {
             if (k < nsub) {
               const uint32_t acc = (kq > 0 || k > 0) ? 1u : 0u;  // the first stage overwrites
-              if constexpr (PAIR)
-                ptx::mma_bf16_pair(d_tmem, adesc + k * A_STEP, bdesc + k * B_STEP, IDESC, acc);
-              else
-                ptx::mma_bf16(d_tmem, adesc + k * A_STEP, bdesc + k * B_STEP, IDESC, acc);
+#pragma unroll
+              for (int h = 0; h < NSPLIT; ++h) {
+                // MMA h reads B columns [128h, 128h+128) of each CTA: 128 x BKM bf16 further
+                // on in either operand layout (two 64-wide chunks, or 128 K-major rows)
+                const uint64_t bh = (uint64_t)h * ((128u * BKM * 2u) >> 4);
+                if constexpr (PAIR)
+                  ptx::mma_bf16_pair(d_tmem + h * MMA_N, adesc + k * A_STEP,
+                                     bdesc + bh + k * B_STEP, IDESC, acc);
+                else
+                  ptx::mma_bf16(d_tmem, adesc + k * A_STEP, bdesc + k * B_STEP, IDESC, acc);
+              }
             }
           }
           // free the stage (in both CTAs of a pair) once these MMAs are done
@@ -766,8 +784,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         continue;
       }
-      const uint32_t a = acc_iter & 1u;
-      if (!warp_wait(&sh.tfull[a], (acc_iter >> 1) & 1u, sh, p, false, GG_EPI_BACKOFF_NS)) break;
+      const uint32_t a = acc_iter % L::ACC_BUFS;
+      if (!warp_wait(&sh.tfull[a], (acc_iter / L::ACC_BUFS) & 1u, sh, p, false,
+                     GG_EPI_BACKOFF_NS))
+        break;
       ptx::tc_fence_after();
       float s_row = 1.f;  // per-row bias scale (read only for rows inside the group)
       if (p.bias != nullptr && p.bias_scale != nullptr && row_ok) s_row = p.bias_scale[orow];
@@ -841,6 +861,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t(&nxt)[32] = ((c / 32) & 1) ? r0 : r1;
         ptx::tmem_ld_wait();
         if (c + 32 < CW) ptx::tmem_ld_32x32b_x32(taddr + c + 32, nxt);
+        // output column of the chunk's first accumulator column: TMEM column t of a 512-wide
+        // pair tile is column 128 (t / 256) + t % 128 of the leader's (t % 256 < 128) or the
+        // follower's B half; narrower tiles map TMEM columns to output columns one to one
+        const int32_t tcol = c_off + c;
+        const int32_t cc = BN > 256 ? tl.n0 + ((tcol % 256) / 128) * L::B_COLS +
+                                          128 * (tcol / 256) + tcol % 128
+                                    : col0 + c;
         if (F32 && row_ok) {
           // fp32 out = alpha * acc + beta * out; the old value is read only when beta != 0.
           // All of the chunk's old values are loaded before the first store, so that the
@@ -852,12 +879,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (p.beta != 0.f) {
 #pragma unroll
             for (int j = 0; j < 8; ++j)
-              if (col0 + c + j * 4 < p.out_cols)
-                old[j] = __ldg(reinterpret_cast<const float4*>(orow_f + col0 + c + j * 4));
+              if (cc + j * 4 < p.out_cols)
+                old[j] = __ldg(reinterpret_cast<const float4*>(orow_f + cc + j * 4));
           }
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const int32_t col = col0 + c + j * 4;
+            const int32_t col = cc + j * 4;
             if (col < p.out_cols) {
               float4 v = make_float4(p.alpha * __uint_as_float(cur[4 * j]),
                                      p.alpha * __uint_as_float(cur[4 * j + 1]),
@@ -873,13 +900,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
         } else if (row_ok) {
-          if (bias_e != nullptr && col0 + c < p.out_cols) {
+          if (bias_e != nullptr && cc < p.out_cols) {
             // h = product + s_row * bias[e, col]; out_cols is a multiple of 8, so a 32-wide
             // chunk is read only up to its last valid 8-column group
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              if (col0 + c + 8 * j < p.out_cols) {
-                const uint4 bv = *reinterpret_cast<const uint4*>(bias_e + col0 + c + 8 * j);
+              if (cc + 8 * j < p.out_cols) {
+                const uint4 bv = *reinterpret_cast<const uint4*>(bias_e + cc + 8 * j);
                 const __nv_bfloat16* bb = reinterpret_cast<const __nv_bfloat16*>(&bv);
 #pragma unroll
                 for (int u = 0; u < 8; ++u)
@@ -898,13 +925,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (v8) {
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-              const int32_t col = col0 + c + j * 16;
+              const int32_t col = cc + j * 16;
               if (col < p.out_cols) ptx::st_global_v8(orow_ptr + col, packed + 8 * j);
             }
           } else {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const int32_t col = col0 + c + j * 8;
+              const int32_t col = cc + j * 8;
               if (col < p.out_cols)
                 *reinterpret_cast<uint4*>(orow_ptr + col) =
                     make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);

@@ -19,9 +19,10 @@ pytestmark = [pytest.mark.gpu,
 gg = pytest.importorskip("moe_grouped_gemm_ragged_b200")
 
 
-@pytest.fixture(params=[1, 2], ids=["single_cta", "cta_pair"])
+@pytest.fixture(params=[1, 2, 3], ids=["single_cta", "cta_pair", "cta_pair_wide"])
 def variant(request):
-    """Run forward/dgrad with 128-row single-CTA tiles and with 256-row CTA-pair tiles."""
+    """Every pass with 128-row single-CTA tiles, 256-row CTA-pair tiles, and CTA pairs
+    with 256 x 512 tiles (the automatic wgrad shape)."""
     prev = gg.testing_force_variant(request.param)
     yield request.param
     gg.testing_force_variant(prev)

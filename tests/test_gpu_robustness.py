@@ -17,7 +17,7 @@ pytestmark = [pytest.mark.gpu,
 gg = pytest.importorskip("moe_grouped_gemm_ragged_b200")
 
 
-@pytest.fixture(params=[1, 2], ids=["single_cta", "cta_pair"])
+@pytest.fixture(params=[1, 2, 3], ids=["single_cta", "cta_pair", "cta_pair_wide"])
 def variant(request):
     prev = gg.testing_force_variant(request.param)
     yield request.param
