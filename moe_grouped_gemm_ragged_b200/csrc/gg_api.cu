@@ -398,7 +398,7 @@ gg_status forward_impl(const void* A, const void* W, const int32_t* offs, void* 
   const bool silu = epi != nullptr && epi->act == GG_ACT_SILU_MUL;
   const bool wnk = (flags & GG_FLAG_W_NK) != 0;
   const bool pair = use_pair(rows_alloc, E);
-  const bool wide = pair && !silu && use_wide(rows_alloc, E, K);
+  const bool wide = pair && use_wide(rows_alloc, E, K);
   const bool chunked = (N % 64) == 0;
   const uint32_t bcols = wide ? kWideBN / 2 : pair ? kBN / 2 : kBN;
   CUtensorMap ma, mb;
@@ -422,7 +422,11 @@ gg_status forward_impl(const void* A, const void* W, const int32_t* offs, void* 
   const int64_t tiles =
       (cdiv(rows_alloc, (pair ? 2 : 1) * gg::BM) + E + 1) * cdiv(N, wide ? kWideBN : kBN);
   if (wide) {
-    if (wnk) return launch<Mode::Dgrad, kWideBN, kWideStages, true>(ma, mb, p, tiles, di, stream);
+    if (wnk) {
+      if (silu) return launch<Mode::Dgrad, kWideBN, kWideStages, true, false, 1>(ma, mb, p, tiles, di, stream);
+      return launch<Mode::Dgrad, kWideBN, kWideStages, true>(ma, mb, p, tiles, di, stream);
+    }
+    if (silu) return launch<Mode::Forward, kWideBN, kWideStages, true, false, 1>(ma, mb, p, tiles, di, stream);
     return launch<Mode::Forward, kWideBN, kWideStages, true>(ma, mb, p, tiles, di, stream);
   }
   if (wnk) {

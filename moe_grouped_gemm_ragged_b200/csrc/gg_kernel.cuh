@@ -795,7 +795,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           p.bias != nullptr ? p.bias + (int64_t)tl.e * p.bias_ld : nullptr;
       if constexpr (ACT == 1) {
         // SiLU-and-mul: this warp owns output columns [oc, oc + CW/2) of the tile; their gate
-        // values are accumulator columns c_off/2 + j and their up values BN/2 further on
+        // values are accumulator columns c_off/2 + j and their up values BN/2 further on. The
+        // gate of accumulator column t < BN/2 is product column 256 (t / 128) + t % 128 and
+        // its up value the column 128 after it (in a 512-wide pair tile the TMEM column
+        // order of the two MMAs puts them there; in a 256-wide tile t < 128)
         const int32_t half = c_off / 2;
         const uint32_t tg = tmem_base + ((q * 32u) << 16) + a * BN + (uint32_t)half;
         const int32_t oc = tl.n0 / 2 + half;
@@ -811,9 +814,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               // gate and up biases of these 32 columns, 8 at a time (16-byte loads)
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
-                const uint4 bg = __ldg(reinterpret_cast<const uint4*>(bias_e + tl.n0 + half + c + 8 * j));
-                const uint4 bu =
-                    __ldg(reinterpret_cast<const uint4*>(bias_e + tl.n0 + BN / 2 + half + c + 8 * j));
+                const int32_t t = half + c + 8 * j;
+                const int32_t gcol = tl.n0 + 256 * (t / 128) + t % 128;
+                const uint4 bg = __ldg(reinterpret_cast<const uint4*>(bias_e + gcol));
+                const uint4 bu = __ldg(reinterpret_cast<const uint4*>(bias_e + gcol + 128));
                 const __nv_bfloat16* g8 = reinterpret_cast<const __nv_bfloat16*>(&bg);
                 const __nv_bfloat16* u8 = reinterpret_cast<const __nv_bfloat16*>(&bu);
 #pragma unroll
