@@ -21,6 +21,7 @@ import json
 import os
 import statistics
 import subprocess
+import threading
 import sys
 import time
 
@@ -124,6 +125,64 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(loaded) if loaded else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
                 "samples": len(rows)}
+
+
+class NvmlClockSampler:
+    """SM clock and clock-event reasons sampled in-process through NVML every 10 ms during
+    the timed region (nvidia-smi, started as a process, catches only a few samples of a
+    region a few hundred milliseconds long). Same summary as ClockSampler.parse."""
+
+    # NVML clock-event reason bits
+    REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        import pynvml
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+        uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+        self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        self.period = period_s
+        self.samples = []
+        self.stop_flag = threading.Event()
+        self.thread = None
+
+    def _run(self):
+        nv = self.nv
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop_flag.is_set():
+            try:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM),
+                                     int(get_reasons(self.h))))
+            except Exception:
+                pass
+            self.stop_flag.wait(self.period)
+
+    def start(self):
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    def stop(self):
+        self.stop_flag.set()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+        if not self.samples:
+            return None
+        sm = [float(c) for c, _ in self.samples]
+        reasons = sorted({name for _, bits in self.samples
+                          for name, bit in self.REASONS.items() if bits & bit})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(self.max_mhz),
+                "reasons": reasons, "samples": len(sm), "source": "nvml, 10 ms"}
+
+
+def make_clock_sampler(device_index: int):
+    try:
+        return NvmlClockSampler(device_index)
+    except Exception:
+        return ClockSampler(device_index)
 
 
 def reduce_max(value: float, device) -> float:
@@ -272,7 +331,7 @@ def run_ours(args):
         raise SystemExit(f"kernel status after warm-up: {[hex(x) for x in st]}")
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    sampler = ClockSampler(local)
+    sampler = make_clock_sampler(local)
     barrier()
     torch.cuda.synchronize()
     sampler.start()

@@ -75,3 +75,18 @@ def test_clock_parser_reports_reasons_and_median():
     assert c["sm_max_mhz"] == 1965.0 and c["reasons"] == ["sw_power_cap"]
     assert c["sm_mhz"] == 1330.0 and c["samples"] == 4
     assert bench.ClockSampler.parse("") is None
+
+
+def test_nvml_sampler_summary_decodes_reason_bits():
+    """The in-process NVML sampler's summary, on samples a fake NVML would return (no GPU):
+    median SM clock, and the clock-event reason bits decoded by name."""
+    s = bench.NvmlClockSampler.__new__(bench.NvmlClockSampler)
+    s.stop_flag = bench.threading.Event()
+    s.thread = None
+    s.max_mhz = 1965
+    s.samples = [(1965, 0x0), (1310, 0x4), (1290, 0x4), (1300, 0x4 | 0x8)]
+    c = s.stop()
+    assert c["sm_mhz"] == 1305.0 and c["sm_max_mhz"] == 1965.0 and c["samples"] == 4
+    assert c["reasons"] == ["hw_slowdown", "sw_power_cap"]
+    s.samples = []
+    assert s.stop() is None
