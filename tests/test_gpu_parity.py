@@ -108,6 +108,17 @@ def test_shuffled_sizes_many_experts(variant):
     check_ragged(r, sample=False)
 
 
+def test_maximum_expert_count(variant):
+    """GG_MAX_EXPERTS = 1024 experts (the largest group tables in shared memory), sizes 0-40
+    rows with a fifth of the experts empty, sampled rows and K rows."""
+    rng = np.random.default_rng(11)
+    sizes = rng.integers(0, 41, 1024)
+    sizes[rng.choice(1024, 205, replace=False)] = 0
+    r = workloads.make_ragged_custom(1024, 128, 192, sizes, seed=12, tail=64)
+    assert r.E == gg.MAX_EXPERTS
+    check_ragged(r, sample=True, seed=5)
+
+
 def test_group_id_probe_bit_exact(variant):
     """A[:,0]=1, W[e][0,:]=e+1: every output row equals its group id + 1 exactly."""
     sizes = [3, 0, 130, 1, 257, 0, 64]
