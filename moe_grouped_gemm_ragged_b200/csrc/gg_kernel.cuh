@@ -668,54 +668,96 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + a * BN;
-        for (int32_t kq = 0; kq < tl.kblocks; ++kq) {
-          const int32_t kb = rev ? tl.kblocks - 1 - kq : kq;
-          if (!wait_bounded(&sh.full[stage], phase, sh, p, true)) { ok = false; break; }
+        // rows of stage kq inside the group: BKM except in a wgrad group's last stage
+        auto rows_of = [&](int32_t kq) {
+          if constexpr (MODE == Mode::Wgrad) {
+            const int32_t kb = rev ? tl.kblocks - 1 - kq : kq;
+            const int32_t rem = tl.tok_len - kb * BKM;
+            return rem < BKM ? rem : BKM;
+          }
+          return BKM;
+        };
+        // waits until stage `st` holds the operands of step kq (false: abort)
+        auto stage_ready = [&](uint32_t st, uint32_t ph, int32_t kq) {
+          if (!wait_bounded(&sh.full[st], ph, sh, p, true)) return false;
 #if GG_FENCE_PER_STAGE
           ptx::tc_fence_after();
 #endif
-          int nsub = BKM / UMMA_K;
-          if constexpr (MODE == Mode::Wgrad) {
-            const int32_t rem = tl.tok_len - kb * BKM;
-            if (rem < BKM) {
-              nsub = (rem + UMMA_K - 1) / UMMA_K;
-              if constexpr (PAIR_WGRAD) {
-                // the follower's half of this stage is fixed up on its own schedule
-                const uint32_t fp = (fixed_par >> stage) & 1u;
-                fixed_par ^= 1u << stage;
-                if (!wait_bounded(&sh.fixed[stage], fp, sh, p, true, true)) { ok = false; break; }
-              }
+          if constexpr (PAIR_WGRAD) {
+            if (rows_of(kq) < BKM) {
+              // a group's last stage: the follower's half is fixed up on its own schedule
+              const uint32_t fp = (fixed_par >> st) & 1u;
+              fixed_par ^= 1u << st;
+              if (!wait_bounded(&sh.fixed[st], fp, sh, p, true, true)) return false;
             }
           }
+          return true;
+        };
+        // the MMAs of accumulator part h (of NSPLIT) for the operands in stage st
+        auto issue = [&](uint32_t st, int32_t kq, int h) {
+          const int nsub = (rows_of(kq) + UMMA_K - 1) / UMMA_K;
           const uint64_t adesc = ptx::smem_desc_sw128(
-              ptx::smem_u32(smem + L::OFF_A + stage * L::A_BYTES), a_lbo, 1024);
-          const uint64_t bdesc = ptx::smem_desc_sw128(
-              ptx::smem_u32(smem + L::OFF_B + stage * L::B_BYTES), b_lbo, 1024);
+              ptx::smem_u32(smem + L::OFF_A + st * L::A_BYTES), a_lbo, 1024);
+          // MMA h reads B columns [128h, 128h+128) of each CTA: 128 x BKM bf16 further on in
+          // either operand layout (two 64-wide chunks, or 128 K-major rows)
+          const uint64_t bdesc =
+              ptx::smem_desc_sw128(ptx::smem_u32(smem + L::OFF_B + st * L::B_BYTES), b_lbo,
+                                   1024) +
+              (uint64_t)h * ((128u * BKM * 2u) >> 4);
 #pragma unroll
           for (int k = 0; k < BKM / UMMA_K; ++k) {
             if (k < nsub) {
               const uint32_t acc = (kq > 0 || k > 0) ? 1u : 0u;  // the first stage overwrites
-#pragma unroll
-              for (int h = 0; h < NSPLIT; ++h) {
-                // MMA h reads B columns [128h, 128h+128) of each CTA: 128 x BKM bf16 further
-                // on in either operand layout (two 64-wide chunks, or 128 K-major rows)
-                const uint64_t bh = (uint64_t)h * ((128u * BKM * 2u) >> 4);
-                if constexpr (PAIR)
-                  ptx::mma_bf16_pair(d_tmem + h * MMA_N, adesc + k * A_STEP,
-                                     bdesc + bh + k * B_STEP, IDESC, acc);
-                else
-                  ptx::mma_bf16(d_tmem, adesc + k * A_STEP, bdesc + k * B_STEP, IDESC, acc);
-              }
+              if constexpr (PAIR)
+                ptx::mma_bf16_pair(d_tmem + h * MMA_N, adesc + k * A_STEP, bdesc + k * B_STEP,
+                                   IDESC, acc);
+              else
+                ptx::mma_bf16(d_tmem, adesc + k * A_STEP, bdesc + k * B_STEP, IDESC, acc);
             }
           }
-          // free the stage (in both CTAs of a pair) once these MMAs are done
+        };
+        // free stage st (in both CTAs of a pair) once the MMAs issued so far are done
+        auto release = [&](uint32_t st) {
           if constexpr (PAIR) {
-            const uint32_t eb = ptx::smem_u32(&sh.empty[stage]);
+            const uint32_t eb = ptx::smem_u32(&sh.empty[st]);
             ptx::mma_commit_pair(ptx::mapa(eb, 0));
             ptx::mma_commit_pair(ptx::mapa(eb, 1));
           } else {
-            ptx::mma_commit(&sh.empty[stage]);
+            ptx::mma_commit(&sh.empty[st]);
           }
+        };
+        int32_t kq = 0;
+        if constexpr (NSPLIT == 2) {
+          // One accumulator in two halves. The epilogue hands the first half back (tempty[0],
+          // waited above) as soon as it holds it in registers, and the second half after
+          // that: the first stages of the tile take their first-half MMAs while the previous
+          // tile's outputs are still being stored, and their second-half MMAs once the second
+          // half is free (tempty[1]); only then are those stages released.
+          const int32_t D = tl.kblocks < STAGES ? tl.kblocks : STAGES;
+          uint32_t st = stage, ph = phase;
+          for (int32_t i = 0; i < D; ++i) {
+            if (!stage_ready(st, ph, i)) { ok = false; break; }
+            issue(st, i, 0);
+            if (++st == STAGES) { st = 0; ph ^= 1u; }
+          }
+          if (!ok) break;
+          if (!wait_bounded(&sh.tempty[1], ((acc_iter / L::ACC_BUFS) & 1u) ^ 1u, sh, p, true,
+                            PAIR)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          for (; kq < D; ++kq) {
+            issue(stage, kq, 1);
+            release(stage);
+            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          }
+        }
+        for (; kq < tl.kblocks; ++kq) {
+          if (!stage_ready(stage, phase, kq)) { ok = false; break; }
+#pragma unroll
+          for (int h = 0; h < NSPLIT; ++h) issue(stage, kq, h);
+          release(stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
@@ -854,6 +896,81 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
         }
+      } else if constexpr (L::ACC_BUFS == 1 && !F32) {
+        // A 512-wide tile in two passes of 128 of this warp's TMEM columns: [0, 256) and then
+        // [256, 512) of the accumulator. A pass takes its columns into registers as bf16,
+        // hands that half of the accumulator back (tempty[pass]) and only then stores them,
+        // so the next tile's MMAs overlap the stores.
+        const int32_t sub = c_off / CW;
+#pragma unroll 1
+        for (int pass = 0; pass < 2; ++pass) {
+          const int32_t tbase = pass * 256 + sub * 128;
+          const uint32_t taddr = tmem_base + ((q * 32u) << 16) + (uint32_t)tbase;
+          // output column of TMEM column t: column 128 (t / 256) + t % 128 of the leader's
+          // (t % 256 < 128) or the follower's B half
+          auto out_col = [&](int32_t t) {
+            return tl.n0 + ((t % 256) / 128) * L::B_COLS + 128 * (t / 256) + t % 128;
+          };
+          uint32_t packed[64];
+          uint32_t r0[32], r1[32];
+          ptx::tmem_ld_32x32b_x32(taddr, r0);
+#pragma unroll
+          for (int c = 0; c < 128; c += 32) {
+            uint32_t(&cur)[32] = ((c / 32) & 1) ? r1 : r0;
+            uint32_t(&nxt)[32] = ((c / 32) & 1) ? r0 : r1;
+            ptx::tmem_ld_wait();
+            if (c + 32 < 128) ptx::tmem_ld_32x32b_x32(taddr + c + 32, nxt);
+            const int32_t cc = out_col(tbase + c);
+            if (bias_e != nullptr && row_ok && cc < p.out_cols) {
+              // h = product + s_row * bias[e, col] (8-column groups up to out_cols)
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                if (cc + 8 * j < p.out_cols) {
+                  const uint4 bv = *reinterpret_cast<const uint4*>(bias_e + cc + 8 * j);
+                  const __nv_bfloat16* bb = reinterpret_cast<const __nv_bfloat16*>(&bv);
+#pragma unroll
+                  for (int u = 0; u < 8; ++u)
+                    cur[8 * j + u] = __float_as_uint(
+                        fmaf(s_row, __bfloat162float(bb[u]), __uint_as_float(cur[8 * j + u])));
+                }
+              }
+            }
+#pragma unroll
+            for (int h = 0; h < 16; ++h) {
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(cur[2 * h]),
+                                                        __uint_as_float(cur[2 * h + 1]));
+              packed[c / 2 + h] = *reinterpret_cast<uint32_t*>(&b2);
+            }
+          }
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if constexpr (PAIR) ptx::mbar_arrive_cluster(pass ? tempty1 : tempty0);
+            else                ptx::mbar_arrive(&sh.tempty[pass]);
+          }
+          if (row_ok) {
+#pragma unroll
+            for (int c = 0; c < 128; c += 32) {
+              const int32_t cc = out_col(tbase + c);
+              if (v8) {
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                  const int32_t col = cc + j * 16;
+                  if (col < p.out_cols) ptx::st_global_v8(orow_ptr + col, packed + c / 2 + 8 * j);
+                }
+              } else {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const int32_t col = cc + j * 8;
+                  if (col < p.out_cols)
+                    *reinterpret_cast<uint4*>(orow_ptr + col) =
+                        make_uint4(packed[c / 2 + 4 * j], packed[c / 2 + 4 * j + 1],
+                                   packed[c / 2 + 4 * j + 2], packed[c / 2 + 4 * j + 3]);
+                }
+              }
+            }
+          }
+        }
       } else {
       const uint32_t taddr = tmem_base + ((q * 32u) << 16) + a * BN + (uint32_t)c_off;
       // 32 columns per load; the next load is in flight while this chunk is stored
@@ -947,8 +1064,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        if constexpr (PAIR) ptx::mbar_arrive_cluster(a ? tempty1 : tempty0);
-        else                ptx::mbar_arrive(&sh.tempty[a]);
+        if constexpr (L::ACC_BUFS == 1) {
+          // one accumulator, handed back in two halves: the register-staged bf16 epilogue
+          // above has released both; the SiLU and fp32 epilogues release both here
+          if constexpr (ACT == 1 || F32) {
+            if constexpr (PAIR) {
+              ptx::mbar_arrive_cluster(tempty0);
+              ptx::mbar_arrive_cluster(tempty1);
+            } else {
+              ptx::mbar_arrive(&sh.tempty[0]);
+              ptx::mbar_arrive(&sh.tempty[1]);
+            }
+          }
+        } else {
+          if constexpr (PAIR) ptx::mbar_arrive_cluster(a ? tempty1 : tempty0);
+          else                ptx::mbar_arrive(&sh.tempty[a]);
+        }
       }
       ++acc_iter;
     }
