@@ -96,7 +96,7 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
-    def stop(self):
+    def stop(self, window=None):
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -155,7 +155,8 @@ class NvmlClockSampler:
             nv.nvmlDeviceGetCurrentClocksThrottleReasons
         while not self.stop_flag.is_set():
             try:
-                self.samples.append((nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM),
+                self.samples.append((time.perf_counter(),
+                                     nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM),
                                      int(get_reasons(self.h))))
             except Exception:
                 pass
@@ -165,14 +166,17 @@ class NvmlClockSampler:
         self.thread = threading.Thread(target=self._run, daemon=True)
         self.thread.start()
 
-    def stop(self):
+    def stop(self, window=None):
+        """Summary of the samples taken inside `window` (perf_counter start, end), or of all."""
         self.stop_flag.set()
         if self.thread is not None:
             self.thread.join(timeout=5)
-        if not self.samples:
+        samples = [x for x in self.samples
+                   if window is None or window[0] <= x[0] <= window[1]]
+        if not samples:
             return None
-        sm = [float(c) for c, _ in self.samples]
-        reasons = sorted({name for _, bits in self.samples
+        sm = [float(c) for _, c, _ in samples]
+        reasons = sorted({name for _, _, bits in samples
                           for name, bit in self.REASONS.items() if bits & bit})
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(self.max_mhz),
                 "reasons": reasons, "samples": len(sm), "source": "nvml, 10 ms"}
@@ -323,6 +327,10 @@ def run_ours(args):
         if evs is not None:
             evs[4].record(stream)
 
+    # NVML samples carry timestamps, so the sampler runs from before the warm-up and only the
+    # samples inside the timed region are kept (no idle gap before the timed steps)
+    sampler = make_clock_sampler(local)
+    sampler.start()
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -331,11 +339,9 @@ def run_ours(args):
         raise SystemExit(f"kernel status after warm-up: {[hex(x) for x in st]}")
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    sampler = make_clock_sampler(local)
     barrier()
     torch.cuda.synchronize()
-    sampler.start()
-    time.sleep(0.3)
+    w0 = time.perf_counter()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
@@ -343,8 +349,9 @@ def run_ours(args):
         step(evs[i])
     t_end.record(stream)
     torch.cuda.synchronize()
+    w1 = time.perf_counter()
     barrier()
-    clocks = sampler.stop()
+    clocks = sampler.stop(window=(w0, w1))
     total_ms = t_start.elapsed_time(t_end)
     per_pass_ms = [sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
                    / args.steps for j in range(4)]

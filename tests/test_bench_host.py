@@ -84,9 +84,12 @@ def test_nvml_sampler_summary_decodes_reason_bits():
     s.stop_flag = bench.threading.Event()
     s.thread = None
     s.max_mhz = 1965
-    s.samples = [(1965, 0x0), (1310, 0x4), (1290, 0x4), (1300, 0x4 | 0x8)]
+    s.samples = [(0.0, 1965, 0x0), (1.0, 1310, 0x4), (2.0, 1290, 0x4), (3.0, 1300, 0x4 | 0x8)]
     c = s.stop()
     assert c["sm_mhz"] == 1305.0 and c["sm_max_mhz"] == 1965.0 and c["samples"] == 4
     assert c["reasons"] == ["hw_slowdown", "sw_power_cap"]
+    # only the samples inside the timed region count
+    c = s.stop(window=(0.5, 2.5))
+    assert c["sm_mhz"] == 1300.0 and c["samples"] == 2 and c["reasons"] == ["sw_power_cap"]
     s.samples = []
     assert s.stop() is None
