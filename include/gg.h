@@ -276,7 +276,10 @@ GG_API gg_status gg_layer_step_host(const void* A_h, const void* W_h, const void
 GG_API const char* gg_status_string(gg_status s);
 
 /* Watchdog bound of every in-kernel wait, in nanoseconds, for later calls from any
-   thread (default 4e9). Returns the previous value. 0 restores the default. */
+   thread (default 4e9). Returns the previous value. 0 restores the default. The longest
+   wait on a healthy call is the epilogue's wait for one tile's whole reduction (K for
+   forward, N for dgrad, a group's rows for wgrad), about 0.5-1 us per 64 reduction
+   elements on a B200: raise the bound for reductions beyond a few million elements. */
 GG_API uint64_t gg_set_watchdog_ns(uint64_t ns);
 
 /* Test hook: when enable != 0, later calls make CTA 0's load warp skip its first stage,
