@@ -7,17 +7,20 @@
 //   Wgrad    dW[e]      = A[rows of e]^T . dY[rows of e] (tile rows = K index; the reduction
 //                                                        runs over the ragged token rows)
 //
-// Two launch shapes share this code:
+// Launch shapes sharing this code:
 //   single CTA (PAIR = false): a tile is 128 rows x BN columns, one CTA per SM;
 //   CTA pair   (PAIR = true):  a cluster of 2 CTAs on neighbouring SMs computes one
 //               256 x BN tile with tcgen05.mma.cta_group::2: each CTA loads its own 128 rows
 //               of A and its own BN/2 columns of B (no multicast), the pair leader issues the
-//               MMAs, and each CTA's tensor memory holds its 128 rows of the accumulator.
+//               MMAs, and each CTA's tensor memory holds its 128 rows of the accumulator;
+//               with BN = 512 (wide pair) each reduction step issues two N = 256 MMAs into
+//               one accumulator of all 512 TMEM columns.
 //
-// Roles of the 6 warps of a CTA (one CTA per SM, persistent over a strided tile list):
+// Roles of the 11 warps of a CTA (one CTA per SM, persistent over a strided tile list):
 //   warp 0      TMA producer: one lane arms a stage barrier and issues the tensor loads
 //   warp 1      tensor-memory owner and MMA issuer: one lane issues tcgen05.mma into a
-//               double-buffered fp32 accumulator in TMEM (2 x BN columns)
+//               double-buffered fp32 accumulator in TMEM (2 x BN columns), or into the single
+//               accumulator of a wide pair, which the epilogue hands back half by half
 //   warps 2..9  epilogue: two warps per 32-lane TMEM quadrant, each owning half of the
 //               columns; tcgen05.ld (double-buffered registers), fp32 -> bf16 (nearest
 //               even), predicated 32- or 16-byte stores of rows inside the group, columns < N
