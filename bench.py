@@ -45,7 +45,7 @@ NCU_TRAFFIC = {
     ("wgrad", "large"): 11.830e9,
     ("masked", "large"): 0.023e9,
 }
-NCU_TRAFFIC_SRC_HASH = "c9234ea399e7b8a5"
+NCU_TRAFFIC_SRC_HASH = "390fc264d1a67214"
 
 
 GEMM_SOURCES = ("gg_kernel.cuh", "ptx.cuh", "gg_api.cu")  # the grouped GEMM kernels + launch
