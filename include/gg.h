@@ -21,6 +21,8 @@
  * memory, pads A or clears an output (TileOPs issue 1566, "Summary": the per-call zero
  * fill and pad cost ~2.8 ms on a ~20 ms GEMM). Every call is ordered on the caller's
  * stream and may be captured in a CUDA graph; the offsets may change between replays.
+ * (gg_layer_step_host, whose operands are host data, is the exception: it reads the
+ * offsets on the host and is not for stream capture; see its description.)
  *
  * Memory. All pointers are device pointers owned by the caller; bf16 arrays are row major
  * (last index contiguous) and 16-byte aligned. W is one packed [E,K,N] buffer (the single
