@@ -24,7 +24,8 @@
  * (gg_layer_step_host, whose operands are host data, is the exception: it reads the
  * offsets on the host and is not for stream capture; see its description.)
  *
- * Memory. All pointers are device pointers owned by the caller; bf16 arrays are row major
+ * Memory. All pointers are device pointers owned by the caller, on the device that is
+ * current when the call is made (the kernels run there); bf16 arrays are row major
  * (last index contiguous) and 16-byte aligned. W is one packed [E,K,N] buffer (the single
  * grouped weight of TransformerEngine PR 3224). K and N must be multiples of 8.
  *
