@@ -201,25 +201,38 @@ gg_status launch(const CUtensorMap& a, const CUtensorMap& b, const gg::Params& p
   }
   int64_t units = tiles_upper < max_units[dev] ? tiles_upper : max_units[dev];
   if (units < 1) units = 1;
-  if (!PAIR) {
-    kern<<<(unsigned)units, gg::NUM_THREADS, smem, stream>>>(a, b, p);
-    ce = cudaGetLastError();
-    return ce == cudaSuccess ? GG_OK : cuda_fail("kernel launch", ce);
-  }
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.gridDim = dim3((unsigned)(2 * units), 1, 1);
+  cudaLaunchAttribute attr[2];
+  unsigned na = 0;
+  if (PAIR) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 2;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  const bool pdl = GG_PDL != 0;
+  if (pdl) {
+    // may start while the previous kernel of the stream finishes (the kernel waits for it
+    // before its first global access)
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.gridDim = dim3((unsigned)(PAIR ? 2 * units : units), 1, 1);
   cfg.blockDim = dim3(gg::NUM_THREADS, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if ((ce = cudaLaunchKernelEx(&cfg, kern, a, b, p)) != cudaSuccess)
-    return cuda_fail("cudaLaunchKernelEx", ce);
+  cfg.numAttrs = na;
+  ce = cudaLaunchKernelEx(&cfg, kern, a, b, p);
+  if (ce != cudaSuccess && pdl) {
+    // a stream or capture that does not take programmatic launches: launch plainly
+    (void)cudaGetLastError();
+    cfg.numAttrs = na - 1;
+    ce = cudaLaunchKernelEx(&cfg, kern, a, b, p);
+  }
+  if (ce != cudaSuccess) return cuda_fail("cudaLaunchKernelEx", ce);
   ce = cudaGetLastError();
   return ce == cudaSuccess ? GG_OK : cuda_fail("kernel launch", ce);
 }

@@ -91,6 +91,12 @@ constexpr int NUM_THREADS = 32 * (FIX_WARP + 1);
 #ifndef GG_EPI_BACKOFF_NS
 #define GG_EPI_BACKOFF_NS 0
 #endif
+// Programmatic dependent launch: a kernel may be scheduled while the previous kernel of its
+// stream is still finishing; it initialises its barriers and tensor memory, then waits for
+// that kernel's completion before its first global read or write (0 launches plainly).
+#ifndef GG_PDL
+#define GG_PDL 1
+#endif
 
 // Device status bits (same values as the public header).
 constexpr int DEV_BAD_OFFSETS = 0x1;
@@ -469,6 +475,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ptx::tmem_relinquish();
     }
   }
+  // Up to here only this CTA's own shared and tensor memory was touched. The inputs may be
+  // the outputs of the previous kernel in the stream, which may still be running.
+  ptx::griddep_wait();
   if (warp == 0) build_table<MODE, BN, TM>(p, sh);
   ptx::tc_fence_before();
   if constexpr (PAIR) ptx::cluster_sync();  // peer barriers initialised before any remote use
@@ -480,6 +489,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
   const uint32_t tmem_base = *sh.tmem_base;
   const int32_t total = *sh.total;
+  // the next kernel may be scheduled on SMs as they free up; it waits for this grid as above
+  ptx::griddep_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
