@@ -37,15 +37,16 @@ UNIT = "TFLOP/s"
 # DRAM bytes per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum), keyed by
 # kernel and workload, valid only for the kernel sources whose hash is recorded with them.
 # Captured with: ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum
-#   --clock-control none -k regex:grouped_gemm -s 12 -c 4 python bench.py --steps 1 --warmup 3
-#   --no-e2e --no-cpu   (see profiles/grouped_gemm_large_launch_list.md)
+#   --clock-control none -k regex:"grouped_gemm|count_kernel|scan_kernel|scatter_kernel"
+#   -s 12 -c 40 python bench.py --steps 1 --warmup 3 --no-e2e --no-cpu  (the first four
+#   captured launches are the timed step; see profiles/grouped_gemm_large_launch_list.md)
 NCU_TRAFFIC = {
-    ("forward", "large"): 9.338e9,
-    ("dgrad", "large"): 10.210e9,
-    ("wgrad", "large"): 11.830e9,
+    ("forward", "large"): 14.396e9,
+    ("dgrad", "large"): 14.195e9,
+    ("wgrad", "large"): 18.248e9,
     ("masked", "large"): 0.023e9,
 }
-NCU_TRAFFIC_SRC_HASH = "390fc264d1a67214"
+NCU_TRAFFIC_SRC_HASH = "ed0f8ba982f4ce4b"
 
 
 GEMM_SOURCES = ("gg_kernel.cuh", "ptx.cuh", "gg_api.cu")  # the grouped GEMM kernels + launch
