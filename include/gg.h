@@ -23,6 +23,11 @@
  * stream and may be captured in a CUDA graph; the offsets may change between replays.
  * (gg_layer_step_host, whose operands are host data, is the exception: it reads the
  * offsets on the host and is not for stream capture; see its description.)
+ * The grouped GEMM kernels are launched with programmatic dependent launch: one may be
+ * scheduled while the kernel before it on the stream is still finishing, and it waits for
+ * that kernel's completion (and its memory) before its first global read or write, so the
+ * stream order above holds for any producer of the inputs. A stream that refuses such a
+ * launch gets a plain one.
  *
  * Memory. All pointers are device pointers owned by the caller, on the device that is
  * current when the call is made (the kernels run there); bf16 arrays are row major
