@@ -32,7 +32,7 @@ gg_status cuda_fail(const char* where, cudaError_t e) {
   return GG_ERR_CUDA;
 }
 std::atomic<int> g_skip_first_load{0};
-// test hook: 0 automatic, 1 single CTA, 2 CTA pair, 3 CTA pair with 512-column wgrad tiles
+// test hook: 0 automatic, 1 single CTA, 2 CTA pair, 3 wide CTA pair (256 x 512 tiles)
 std::atomic<int> g_force_variant{0};
 
 static_assert(gg::DEV_BAD_OFFSETS == GG_DEV_BAD_OFFSETS, "status bit mismatch");
