@@ -11,8 +11,9 @@
 //   single CTA (PAIR = false): a tile is 128 rows x BN columns, one CTA per SM;
 //   CTA pair   (PAIR = true):  a cluster of 2 CTAs on neighbouring SMs computes one
 //               256 x BN tile with tcgen05.mma.cta_group::2: each CTA loads its own 128 rows
-//               of A and its own BN/2 columns of B (no multicast), the pair leader issues the
-//               MMAs, and each CTA's tensor memory holds its 128 rows of the accumulator;
+//               of A and its own BN/2 columns of B into its own shared memory, the pair
+//               leader issues the MMAs, and each CTA's tensor memory holds its 128 rows of
+//               the accumulator;
 //               with BN = 512 (wide pair) each reduction step issues two N = 256 MMAs into
 //               one accumulator of all 512 TMEM columns.
 //
