@@ -119,8 +119,8 @@ def testing_skip_first_load(enable: bool) -> bool:
 
 
 def testing_force_variant(variant: int) -> int:
-    """Test hook: 0 automatic, 1 single-CTA tiles, 2 CTA-pair tiles (forward, dgrad, wgrad),
-    3 CTA pairs with 256 x 512 tiles (the automatic wgrad shape)."""
+    """Test hook: 0 automatic, 1 single-CTA tiles, 2 CTA-pair tiles, 3 wide CTA pairs
+    (256 x 512 tiles, the automatic shape of long reductions), each for every pass."""
     return int(lib().gg_testing_force_variant(int(variant)))
 
 
