@@ -34,22 +34,17 @@ import torch  # noqa: E402
 METRIC = "grouped GEMM BF16 TFLOP/s (fwd/dgrad/wgrad) and % of B200 dense BF16 peak"
 UNIT = "TFLOP/s"
 
-# DRAM bytes per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum), keyed by
-# kernel and workload, valid only for the kernel sources whose hash is recorded with them.
-# Captured with: ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum
-#   --clock-control none -k regex:"grouped_gemm|count_kernel|scan_kernel|scatter_kernel"
-#   -s 12 -c 40 python bench.py --steps 1 --warmup 3 --no-e2e --no-cpu  (the first four
-#   captured launches are the timed step; see profiles/grouped_gemm_large_launch_list.md)
-NCU_TRAFFIC = {
-    ("forward", "large"): 14.396e9,
-    ("dgrad", "large"): 14.195e9,
-    ("wgrad", "large"): 18.248e9,
-    ("masked", "large"): 0.023e9,
-}
-NCU_TRAFFIC_SRC_HASH = "7646bde52dacab86"
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant kernel,
+# keyed by pass and workload, valid only for the kernel sources whose hash is recorded with
+# them (a changed kernel reports null until it is captured again). Each figure comes from a
+# capture of ONE launch of ONE kernel (-k <kernel> -c 1) with only these counters, which ncu
+# collects in a single pass; a launch list over many kernels collects gpu__time_duration.sum
+# alone.
+NCU_TRAFFIC = {}
+NCU_TRAFFIC_SRC_HASH = ""
 
 
-GEMM_SOURCES = ("gg_kernel.cuh", "ptx.cuh", "gg_api.cu")  # the grouped GEMM kernels + launch
+GEMM_SOURCES = ("gg_kernel.cuh", "ptx.cuh", "gg_api.cu", "gg_masked.cuh")  # kernels + launch
 
 
 def kernel_source_hash() -> str:
@@ -361,8 +356,15 @@ def run_ours(args):
     value = ws * step_flops / (ms_per_step * 1e-3) / 1e12
 
     extras = None
+    peaks, peak_src = load_peaks()
     if not args.no_extras:
         extras = run_extras(args, gg, r, dev, stream, offs, out, dW)
+        extras["masked"] = masked_timings(gg, m, dev, peaks)
+        extras["masked"]["ms_in_step"] = per_pass_ms[3]
+        extras["tiny_forward_call"] = tiny_call_costs(gg, dev)
+        if ws == 1:
+            extras["configs"] = run_config_extras(gg, dev, stream, peaks,
+                                                  reps=max(5, args.steps))
 
     # end to end through the public API: pinned host inputs -> device, all passes, results
     # back to pinned host memory, every step inside the timed region
@@ -370,7 +372,6 @@ def run_ours(args):
     if not args.no_e2e:
         e2e = run_e2e(args, gg, r, m, dev, stream, ws, barrier)
 
-    peaks, peak_src = load_peaks()
     dom = int(np.argmax(per_pass_ms[:3]))
     dom_tflops = pass_flops[dom] / (per_pass_ms[dom] * 1e-3) / 1e12
     peak_sus = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
@@ -475,6 +476,115 @@ def run_extras(args, gg, r, dev, stream, offs, out, dW):
         else:
             res[name] = {"ms": ms, "tflops": r.flops / (ms * 1e-3) / 1e12, "launches": reps}
     return res
+
+
+def run_config_extras(gg, dev, stream, peaks, reps: int):
+    """Forward, dgrad and wgrad of the other ragged configs (gate-up E=64 Zipf, down-proj E=32,
+    the large shape with unaligned sizes), each pass timed on its own outside the step: median
+    of per-call CUDA-event times of `reps` back-to-back calls after 3 warm-up calls."""
+    import workloads
+    res = {}
+    for name in ("gateup", "downproj", "large_unaligned"):
+        r = workloads.make_ragged(name, tail=0, device=dev)
+        offs = torch.from_numpy(r.offs).to(dev)
+        out = torch.empty((r.rows_alloc, r.N), dtype=torch.bfloat16, device=dev)
+        dX = torch.empty((r.rows_alloc, r.K), dtype=torch.bfloat16, device=dev)
+        dW = torch.empty((r.E, r.K, r.N), dtype=torch.bfloat16, device=dev)
+        fns = {"forward": lambda: gg.forward(r.A, r.W, offs, out),
+               "dgrad": lambda: gg.dgrad(r.dY, r.W, offs, dX),
+               "wgrad": lambda: gg.wgrad(r.A, r.dY, offs, dW)}
+        entry = {"E": r.E, "T": r.T, "K": r.K, "N": r.N, "flops_per_pass": r.flops,
+                 "group_sizes": f"min {int(r.sizes.min())} max {int(r.sizes.max())}, "
+                                f"{int((r.sizes == 0).sum())} empty"}
+        for pas, fn in fns.items():
+            ms = _median_call_ms(fn, stream, reps)
+            tf = r.flops / (ms * 1e-3) / 1e12
+            entry[pas] = {"ms": ms, "tflops": tf, "frac_of_burst": tf / peaks["bf16_tflops"]}
+        res[name] = entry
+        del r, offs, out, dX, dW, fns
+        torch.cuda.empty_cache()
+    return res
+
+
+def masked_timings(gg, m, dev, peaks, copies: int = 16, rounds: int = 12):
+    """Per-call time of the masked forward replayed from a CUDA graph: `hot` calls reuse one
+    set of inputs (the weights stay in L2), `cold` calls cycle through `copies` sets of inputs
+    (copies x 25 MB, above the 126 MB L2), so every call reads its weights from HBM."""
+    mm = torch.from_numpy(m.masked_m).to(dev)
+    As = [m.A] + [m.A.clone() for _ in range(copies - 1)]
+    Ws = [m.W] + [m.W.clone() for _ in range(copies - 1)]
+    outs = [torch.empty((m.E, m.mmax, m.N), dtype=torch.bfloat16, device=dev)
+            for _ in range(copies)]
+    side = torch.cuda.Stream(device=dev)
+
+    def per_call_us(seq):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            for i in seq:
+                gg.masked_forward(As[i], Ws[i], mm, outs[i])
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        cur = torch.cuda.current_stream(dev)
+        a.record(cur)
+        g.replay()
+        b.record(cur)
+        torch.cuda.synchronize()
+        del g
+        return a.elapsed_time(b) * 1e3 / len(seq)
+
+    gg.masked_forward(As[0], Ws[0], mm, outs[0])
+    torch.cuda.synchronize()
+    hot = float(np.median([per_call_us([0] * 200) for _ in range(3)]))
+    cold = float(np.median([per_call_us(list(range(copies)) * rounds) for _ in range(3)]))
+    nbytes = masked_bytes(m)
+    return {"algorithmic_bytes": nbytes, "hot_graph_us": hot, "cold_graph_us": cold,
+            "cold_gbs": nbytes / (cold * 1e-6) / 1e9,
+            "cold_frac_of_hbm": nbytes / (cold * 1e-6) / 1e9 / peaks["hbm_gbs"],
+            "hot_gbs": nbytes / (hot * 1e-6) / 1e9,
+            "kernel": "masked_forward_kernel (weight columns as the MMA's M)"}
+
+
+def tiny_call_costs(gg, dev, calls: int = 2000):
+    """Cost of one call of the tiny forward (4 experts, A[48, 8], offsets (8,16,32,40)), the
+    shape where the host launch dominates: host time per call through the Python binding and
+    through the C ABI alone (ctypes, arguments prepared once), CUDA-event time per call of
+    back-to-back calls, and the per-call time of calls replayed from a CUDA graph."""
+    import time as _t
+    import workloads
+    r = workloads.make_tiny((8, 16, 32, 40))
+    A, W = r.A.to(dev), r.W.to(dev)
+    offs = torch.from_numpy(np.ascontiguousarray(r.offs)).to(dev)
+    out = torch.empty((r.rows_alloc, r.N), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    fn = lambda: gg.forward(A, W, offs, out)  # noqa: E731
+    L = gg.lib()
+    cargs = (A.data_ptr(), W.data_ptr(), offs.data_ptr(), out.data_ptr(), r.rows_alloc, r.K,
+             r.N, r.E, None, stream.cuda_stream)
+    cfn = L.gg_forward
+
+    def host_us(f):
+        for _ in range(50):
+            f()
+        torch.cuda.synchronize()
+        t0 = _t.perf_counter()
+        for _ in range(calls):
+            f()
+        t1 = _t.perf_counter()
+        torch.cuda.synchronize()
+        return (t1 - t0) * 1e6 / calls
+
+    py = host_us(fn)
+    cabi = host_us(lambda: cfn(*cargs))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(calls):
+        cfn(*cargs)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return {"host_us_python_binding": py, "host_us_c_abi": cabi,
+            "event_us_back_to_back_c_abi": e0.elapsed_time(e1) * 1e3 / calls,
+            "graph_us": _graph_call_us(fn, stream, 200), "calls": calls}
 
 
 def run_e2e(args, gg, r, m, dev, stream, ws, barrier):
@@ -663,11 +773,16 @@ def run_table(args):
     mout = torch.empty((m.E, m.mmax, m.N), dtype=torch.bfloat16, device=dev)
     fn = lambda: gg.masked_forward(mA, mW, mm, mout)  # noqa: E731
     ms = _median_call_ms(fn, stream, 200)
-    gus = _graph_call_us(fn, stream, 200)
+    mt = masked_timings(gg, m, dev, peaks)
     t0 = time.perf_counter()
     oracle.masked_forward(oracle.as_u16(mA), oracle.as_u16(mW), m.masked_m, threads=threads)
     osec = time.perf_counter() - t0
-    emit("masked", "forward", m.flops, masked_bytes(m), ms, osec, "full pass", gus)
+    # graph-replayed per call with the weights read from HBM (16 rotating input copies)
+    emit("masked", "forward", m.flops, masked_bytes(m), ms, osec, "full pass",
+         mt["cold_graph_us"])
+    print(json.dumps({"config": "masked", "pass": "forward", "graph_timings": mt}), flush=True)
+    print(json.dumps({"config": "tiny (8,16,32,40)", "pass": "forward",
+                      "call_costs": tiny_call_costs(gg, dev)}), flush=True)
     return 0
 
 

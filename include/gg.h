@@ -242,9 +242,12 @@ GG_API gg_status gg_route(const int32_t* topk_ids, int64_t T_tok, int32_t k, int
  * return GG_ERR_TOO_LARGE (e.g. at most 65536 assignments with 1024 experts, 1048576 with
  * 64). Nothing is allocated, freed or cleared: every entry a call reads it wrote itself.
  * All calls share the array, so calls that overlap on the GPU (other streams, other threads)
- * race; order them on one stream. The first call on a device looks up the array's device
- * address (cudaGetSymbolAddress) with that device current; make that first call before any
- * stream capture.
+ * race; order them on one stream. Calls captured in a CUDA graph count the same way: two
+ * replays of such a graph that may run at the same time, or two captured calls on parallel
+ * branches of one graph, overlap and race, so serialise them like calls on two streams.
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ * that device current, and so does the first call after its context was destroyed and
+ * created again (cudaDeviceReset); make such a call before any stream capture.
  */
 #define GG_ROUTE_NOALLOC_MAX_COUNTS (1 << 18)
 GG_API gg_status gg_route_noalloc(const int32_t* topk_ids, int64_t T_tok, int32_t k, int32_t E,

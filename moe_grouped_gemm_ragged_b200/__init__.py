@@ -133,6 +133,10 @@ def _stream_handle(stream) -> int:
 
 
 def _check(t: torch.Tensor, name: str, dtype, ndim: int):
+    # fast path: one combined test; the message below names the first failing property
+    if (isinstance(t, torch.Tensor) and t.dtype is dtype and t.dim() == ndim and t.is_cuda
+            and t.is_contiguous() and t.get_device() == torch.cuda.current_device()):
+        return
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
     if t.device.type != "cuda":

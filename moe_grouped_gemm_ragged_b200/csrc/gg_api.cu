@@ -14,6 +14,7 @@
 
 #include "gg.h"
 #include "gg_kernel.cuh"
+#include "gg_masked.cuh"
 
 namespace {
 
@@ -55,13 +56,34 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 struct DeviceInfo {
+  int dev = 0;
   int sms = 0;
   bool sm100 = false;
-  bool ready = false;
 };
 
-DeviceInfo g_dev[kMaxDevices];
+// Per device: filled once (under the mutex), then read without locking.
+struct DeviceSlot {
+  std::atomic<bool> ready{false};
+  int sms = 0;
+  bool sm100 = false;
+};
+DeviceSlot g_dev[kMaxDevices];
 std::mutex g_dev_mu;
+
+// Driver entry point that tells whether the calling thread has a current context.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(ptr);
+  });
+  return fn;
+}
 
 gg_status device_info(DeviceInfo* out) {
   int dev = 0;
@@ -69,29 +91,84 @@ gg_status device_info(DeviceInfo* out) {
   if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
   if (dev < 0 || dev >= kMaxDevices) return GG_ERR_UNSUPPORTED;
   // Tensor maps are encoded with a driver call, which needs a current context; a thread
-  // that has not touched CUDA yet (e.g. an autograd worker) may have none.
-  if ((e = cudaSetDevice(dev)) != cudaSuccess) return cuda_fail("cudaSetDevice", e);
-  std::lock_guard<std::mutex> lk(g_dev_mu);
-  DeviceInfo& d = g_dev[dev];
-  if (!d.ready) {
-    int major = 0, minor = 0, sms = 0;
-    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
-        (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
-        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
-      return cuda_fail("cudaDeviceGetAttribute", e);
-    d.sms = sms;
-    d.sm100 = (major == 10 && minor == 0);
-    d.ready = true;
+  // that has not touched CUDA yet (e.g. an autograd worker) may have none, and then the
+  // device is made current (which creates its primary context).
+  CUcontext ctx = nullptr;
+  auto get_current = ctx_get_current_fn();
+  if (get_current == nullptr || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr)
+    if ((e = cudaSetDevice(dev)) != cudaSuccess) return cuda_fail("cudaSetDevice", e);
+  DeviceSlot& d = g_dev[dev];
+  if (!d.ready.load(std::memory_order_acquire)) {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!d.ready.load(std::memory_order_relaxed)) {
+      int major = 0, minor = 0, sms = 0;
+      if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+          (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+          (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return cuda_fail("cudaDeviceGetAttribute", e);
+      d.sms = sms;
+      d.sm100 = (major == 10 && minor == 0);
+      d.ready.store(true, std::memory_order_release);
+    }
   }
-  *out = d;
+  out->dev = dev;
+  out->sms = d.sms;
+  out->sm100 = d.sm100;
   return GG_OK;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Recently encoded tensor maps of this thread. A map is a pure function of its description
+// (address, sizes, strides, box), so a cached one stays valid whatever the memory holds;
+// repeated calls on the same buffers skip the encoding.
+struct MapKey {
+  const void* base;
+  int rank;
+  uint64_t dims[4];
+  uint64_t strides[3];
+  uint32_t box[4];
+};
+struct MapCache {
+  static constexpr int kSlots = 16;
+  MapKey key[kSlots];
+  CUtensorMap map[kSlots];
+  int used = 0;
+  int next = 0;  // slot replaced next (round robin)
+};
+thread_local MapCache t_maps;
+
+bool make_map_uncached(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                       const uint64_t* strides_bytes, const uint32_t* box);
+
 // Tiled bf16 tensor map with 128-byte swizzle; out-of-range elements read as zero.
 bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
               const uint64_t* strides_bytes, const uint32_t* box) {
+  MapKey k;
+  std::memset(&k, 0, sizeof(k));
+  k.base = base;
+  k.rank = rank;
+  for (int i = 0; i < rank; ++i) {
+    k.dims[i] = dims[i];
+    k.box[i] = box[i];
+  }
+  for (int i = 0; i + 1 < rank; ++i) k.strides[i] = strides_bytes[i];
+  MapCache& c = t_maps;
+  for (int i = 0; i < c.used; ++i)
+    if (std::memcmp(&c.key[i], &k, sizeof(k)) == 0) {
+      *m = c.map[i];
+      return true;
+    }
+  if (!make_map_uncached(m, base, rank, dims, strides_bytes, box)) return false;
+  const int slot = c.used < MapCache::kSlots ? c.used++ : c.next;
+  if (c.used == MapCache::kSlots) c.next = (slot + 1) % MapCache::kSlots;
+  c.key[slot] = k;
+  c.map[slot] = *m;
+  return true;
+}
+
+bool make_map_uncached(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                       const uint64_t* strides_bytes, const uint32_t* box) {
   auto fn = encode_fn();
   if (fn == nullptr) {
     snprintf(g_err, sizeof(g_err), "cuTensorMapEncodeTiled: driver entry point not found");
@@ -162,15 +239,16 @@ gg_status launch(const CUtensorMap& a, const CUtensorMap& b, const gg::Params& p
   auto kern = gg::grouped_gemm_kernel<MODE, BN, STAGES, PAIR, F32, ACT>;
   using L = gg::Layout<BN, STAGES, PAIR, gg::bk_of<MODE>()>;
   const size_t smem = L::bytes(p.E);
-  int dev = 0;
-  cudaError_t ce = cudaGetDevice(&dev);
-  if (ce != cudaSuccess) return cuda_fail("cudaGetDevice", ce);
-  static bool attr_done[kMaxDevices] = {};
+  const int dev = di.dev;
+  cudaError_t ce = cudaSuccess;
+  // per device, once: the shared-memory attribute and the resident units (read without a
+  // lock afterwards)
+  static std::atomic<bool> attr_done[kMaxDevices];
   static int max_units[kMaxDevices] = {};
   static std::mutex mu;
-  {
+  if (!attr_done[dev].load(std::memory_order_acquire)) {
     std::lock_guard<std::mutex> lk(mu);
-    if (!attr_done[dev]) {
+    if (!attr_done[dev].load(std::memory_order_relaxed)) {
       const int max_smem = (int)L::bytes(GG_MAX_EXPERTS);
       if ((ce = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      max_smem)) != cudaSuccess)
@@ -196,7 +274,7 @@ gg_status launch(const CUtensorMap& a, const CUtensorMap& b, const gg::Params& p
         units = clusters;
       }
       max_units[dev] = units;
-      attr_done[dev] = true;
+      attr_done[dev].store(true, std::memory_order_release);
     }
   }
   int64_t units = tiles_upper < max_units[dev] ? tiles_upper : max_units[dev];
@@ -277,7 +355,6 @@ int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 constexpr int kBN = 256;
 constexpr int kStages = 4;      // single CTA: 48 KB per stage
 constexpr int kPairStages = 6;  // CTA pair: 32 KB per stage and CTA
-constexpr int kMaskedBN = 128;  // masked forward: 128 x 128 tiles, 32 KB per stage
 constexpr int kWgBK = gg::bk_of<Mode::Wgrad>();  // token rows per wgrad stage
 constexpr int kWgStages = kStages;
 constexpr int kWgPairStages = kPairStages;
@@ -507,6 +584,95 @@ gg_status dgrad_impl(const void* dY, const void* W, const int32_t* offs, void* d
   return launch<Mode::Dgrad, kBN, kStages, false>(ma, mb, p, tiles, di, stream);
 }
 
+// Launch of the masked forward kernel (weight columns as the MMA's M): one CTA per SM at
+// most, no cluster, programmatic dependent launch as in launch().
+template <int SW, int ST>
+gg_status launch_masked(const CUtensorMap& mw, const CUtensorMap (&mt)[3],
+                        const gg::masked::Params& p, int64_t units, int dev,
+                        cudaStream_t stream) {
+  auto kern = gg::masked::masked_forward_kernel<SW, ST>;
+  using L = gg::masked::Layout<SW, ST>;
+  static_assert(L::bytes(GG_MAX_EXPERTS) <= 227 * 1024, "shared memory of a CTA exceeded");
+  cudaError_t ce = cudaSuccess;
+  static std::atomic<bool> attr_done[kMaxDevices];
+  static std::mutex mu;
+  if (!attr_done[dev].load(std::memory_order_acquire)) {
+    std::lock_guard<std::mutex> lk(mu);
+    if (!attr_done[dev].load(std::memory_order_relaxed)) {
+      if ((ce = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)L::bytes(GG_MAX_EXPERTS))) != cudaSuccess)
+        return cuda_fail("cudaFuncSetAttribute", ce);
+      attr_done[dev].store(true, std::memory_order_release);
+    }
+  }
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3((unsigned)units, 1, 1);
+  cfg.blockDim = dim3(gg::masked::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = L::bytes(p.E);
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = GG_PDL != 0 ? 1 : 0;
+  ce = cudaLaunchKernelEx(&cfg, kern, mw, mt[0], mt[1], mt[2], p);
+  if (ce != cudaSuccess && cfg.numAttrs == 1) {
+    (void)cudaGetLastError();
+    cfg.numAttrs = 0;
+    ce = cudaLaunchKernelEx(&cfg, kern, mw, mt[0], mt[1], mt[2], p);
+  }
+  if (ce != cudaSuccess) return cuda_fail("cudaLaunchKernelEx", ce);
+  ce = cudaGetLastError();
+  return ce == cudaSuccess ? GG_OK : cuda_fail("kernel launch", ce);
+}
+
+// Weight and token stages of the masked forward kernel, 16 KB each: a reduction step needs
+// one of each (6 + 6, 7 + 5, 5 + 7 and 8 + 4 measured within 2% of one another on the
+// sglang shape).
+constexpr int kMaskedWStages = 6;
+constexpr int kMaskedTStages = 6;
+
+// Masked forward without an activation: the small-batch kernel of gg_masked.cuh (bias and
+// per-row bias scale fused; checked as in set_epilogue).
+gg_status masked_small_impl(const void* A, const void* W, const int32_t* masked_m, void* out,
+                            int64_t mmax, int64_t K, int64_t N, int32_t E,
+                            const gg_epilogue* epi, int32_t* dev_status, const DeviceInfo& di,
+                            cudaStream_t stream) {
+  gg::Params chk;
+  std::memset(&chk, 0, sizeof(chk));
+  gg_status s = set_epilogue(&chk, epi, N);
+  if (s != GG_OK) return s;
+  CUtensorMap mw, mt[3];
+  const bool chunked = (N % 64) == 0;
+  if (chunked ? !map_w_chunked(&mw, W, E, K, N, gg::masked::KBLK, 2)
+              : !map_w(&mw, W, E, K, N, 64, gg::masked::KBLK))
+    return GG_ERR_CUDA;
+  // token rows in boxes of 32, 64 and 128 rows: one or two boxes cover a block's active rows
+  for (int i = 0; i < 3; ++i)
+    if (!map_2d(&mt[i], A, (int64_t)E * mmax, K, gg::masked::KBLK, 32u << i)) return GG_ERR_CUDA;
+  gg::masked::Params p;
+  std::memset(&p, 0, sizeof(p));
+  p.masked_m = masked_m;
+  p.out = reinterpret_cast<__nv_bfloat16*>(out);
+  p.status = dev_status;
+  p.bias = chk.bias;
+  p.bias_scale = chk.bias_scale;
+  p.E = E;
+  p.mmax = (int32_t)mmax;
+  p.K = (int32_t)K;
+  p.N = (int32_t)N;
+  p.watchdog_ns = g_watchdog_ns.load();
+  p.debug_flags = g_skip_first_load.load() ? 1 : 0;
+  p.w_chunked = chunked ? 1 : 0;
+  // every (expert, row block, column tile), active or not; when each can have a CTA of its
+  // own, the CTAs need no tile table (one-tile schedule)
+  const int64_t tiles = (int64_t)E * cdiv(mmax, gg::masked::TILE_T) * cdiv(N, gg::masked::TILE_N);
+  p.one_tile = tiles <= di.sms ? 1 : 0;
+  const int64_t units = tiles < di.sms ? tiles : di.sms;
+  return launch_masked<kMaskedWStages, kMaskedTStages>(mw, mt, p, units < 1 ? 1 : units, di.dev,
+                                                       stream);
+}
+
 gg_status masked_impl(const void* A, const void* W, const int32_t* masked_m, void* out,
                       int64_t mmax, int64_t K, int64_t N, int32_t E, const gg_epilogue* epi,
                       int32_t* dev_status, cudaStream_t stream) {
@@ -519,12 +685,13 @@ gg_status masked_impl(const void* A, const void* W, const int32_t* masked_m, voi
   if (mmax == 0) return GG_OK;
   if (A == nullptr || out == nullptr) return GG_ERR_INVALID_ARG;
   if (!aligned16(A) || !aligned16(W) || !aligned16(out)) return GG_ERR_UNSUPPORTED;
-  // A handful of experts with at most mmax rows each: narrower N-tiles spread the weight
-  // reads (the whole cost of this memory-bound shape) over more SMs, and A is fetched in
-  // 32-row boxes covering only the active rows. SiLU-and-mul needs gate and up columns in
-  // one tile, so it keeps 256-wide tiles.
   const bool silu = epi != nullptr && epi->act == GG_ACT_SILU_MUL;
-  const int bn = silu ? kBN : kMaskedBN;
+  if (!silu)
+    return masked_small_impl(A, W, masked_m, out, mmax, K, N, E, epi, dev_status, di, stream);
+  // SiLU-and-mul needs the gate and up columns of a row in one tile: token rows as the MMA's
+  // M, 256-wide column tiles (gate and up blocks of 128), A fetched in 32-row boxes covering
+  // only the active rows.
+  const int bn = kBN;
   const bool chunked = (N % 64) == 0;
   CUtensorMap ma, mb;
   if (!map_2d(&ma, A, (int64_t)E * mmax, K, 64, 32)) return GG_ERR_CUDA;
@@ -540,8 +707,7 @@ gg_status masked_impl(const void* A, const void* W, const int32_t* masked_m, voi
   p.prod_cols = (int32_t)N;
   set_store_width(&p, out, out_cols);
   const int64_t tiles = (int64_t)E * cdiv(mmax, gg::BM) * cdiv(N, bn);
-  if (silu) return launch<Mode::Masked, kBN, kStages, false, false, 1>(ma, mb, p, tiles, di, stream);
-  return launch<Mode::Masked, kMaskedBN, kPairStages, false>(ma, mb, p, tiles, di, stream);
+  return launch<Mode::Masked, kBN, kStages, false, false, 1>(ma, mb, p, tiles, di, stream);
 }
 
 }  // namespace

@@ -6,11 +6,22 @@
 #include <cstring>
 #include <mutex>
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "gg.h"
 
 namespace ggr {
+
+// The library is built for sm_100a only: the device must be compute capability 10.0 exactly.
+gg_status check_device() {
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return GG_ERR_CUDA;
+  return (major == 10 && minor == 0) ? GG_OK : GG_ERR_UNSUPPORTED;
+}
 
 constexpr int THREADS = 256;          // one assignment per thread and block
 constexpr int WARPS = THREADS / 32;
@@ -204,11 +215,8 @@ gg_status gg_route(const int32_t* topk_ids, int64_t T_tok, int32_t k, int32_t E,
       mis(X, 16) || mis(A_packed, 16) || (dev_status != nullptr && mis(dev_status, 4)))
     return GG_ERR_UNSUPPORTED;
   if (workspace_bytes < gg_route_workspace_bytes(n, E)) return GG_ERR_INVALID_ARG;
-  int dev = 0, major = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
-    return GG_ERR_CUDA;
-  if (major != 10) return GG_ERR_UNSUPPORTED;
+  const gg_status ds = check_device();
+  if (ds != GG_OK) return ds;
   const int64_t nblk = blocks_for(n);
   int32_t* counts = reinterpret_cast<int32_t*>(workspace);
   if (nblk > 0)
@@ -234,29 +242,64 @@ gg_status gg_route(const int32_t* topk_ids, int64_t T_tok, int32_t k, int32_t E,
 // allocator, or code that must not enter the CUDA allocator at that point). Its per-block
 // histograms live in this fixed array instead of a caller-provided workspace. Every GPU that
 // loads the library holds the array (1 MiB) until the process exits. Host code only sees a
-// stand-in for it, so its device address is looked up once per device with
-// cudaGetSymbolAddress while that device is current.
+// stand-in for it, so its device address is looked up with cudaGetSymbolAddress while the
+// device is current: once per device and context (a context that is destroyed and created
+// again, e.g. after cudaDeviceReset, reloads the module, and the array may move).
 static __device__ __align__(256) int32_t g_route_counts[GG_ROUTE_NOALLOC_MAX_COUNTS];
 
 namespace ggr {
 
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
-int32_t* g_noalloc_counts[kMaxDevices] = {};
+struct NoallocSlot {
+  int32_t* counts = nullptr;
+  unsigned long long ctx_id = 0;  // context the address belongs to
+};
+NoallocSlot g_noalloc[kMaxDevices];
 
-// Device address of g_route_counts on the current device (looked up on first use).
+// Unique id of the calling thread's current context (driver entry points, no link to the
+// driver library); 0 when there is none or it cannot be read.
+unsigned long long current_ctx_id() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrent>(f);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(f);
+  });
+  CUcontext c = nullptr;
+  unsigned long long id = 0;
+  if (get_current == nullptr || get_id == nullptr || get_current(&c) != CUDA_SUCCESS ||
+      c == nullptr || get_id(c, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of g_route_counts on the current device, looked up on the first call in
+// each context.
 gg_status noalloc_counts(int32_t** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return GG_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return GG_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (g_noalloc_counts[dev] == nullptr) {
+  NoallocSlot& slot = g_noalloc[dev];
+  const unsigned long long ctx = current_ctx_id();
+  if (slot.counts == nullptr || ctx == 0 || ctx != slot.ctx_id) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_route_counts) != cudaSuccess || p == nullptr)
       return GG_ERR_CUDA;
-    g_noalloc_counts[dev] = static_cast<int32_t*>(p);
+    slot.counts = static_cast<int32_t*>(p);
+    slot.ctx_id = current_ctx_id();  // the lookup made the device's context current
   }
-  *out = g_noalloc_counts[dev];
+  *out = slot.counts;
   return GG_OK;
 }
 
@@ -285,11 +328,8 @@ gg_status gg_route_noalloc(const int32_t* topk_ids, int64_t T_tok, int32_t k, in
   if (mis(topk_ids, 4) || mis(row_of, 4) || mis(offs, 4) || mis(X, 16) || mis(A_packed, 16) ||
       (dev_status != nullptr && mis(dev_status, 4)))
     return GG_ERR_UNSUPPORTED;
-  int dev = 0, major = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
-    return GG_ERR_CUDA;
-  if (major != 10) return GG_ERR_UNSUPPORTED;
+  const gg_status ds = check_device();  // before the symbol is touched or anything launches
+  if (ds != GG_OK) return ds;
   int32_t* counts = nullptr;
   const gg_status s = noalloc_counts(&counts);
   if (s != GG_OK) return s;

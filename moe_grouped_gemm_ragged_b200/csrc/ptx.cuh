@@ -105,6 +105,24 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const void* tmap, uint64_
       : "memory");
 }
 
+// Prefetch of one tensor box into L2 (no shared memory, no barrier). It only warms the cache:
+// L2 is the point of coherence of device memory, so it may run before the grid dependency is
+// resolved without reading anything the previous kernel writes later.
+__device__ __forceinline__ void tma_prefetch_l2_3d(const void* tmap, int32_t x, int32_t y,
+                                                   int32_t z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(tmap)),
+               "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_l2_4d(const void* tmap, int32_t x, int32_t y,
+                                                   int32_t z, int32_t w) {
+  asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                   reinterpret_cast<uint64_t>(tmap)),
+               "r"(x), "r"(y), "r"(z), "r"(w)
+               : "memory");
+}
+
 // L2 eviction-priority policies (createpolicy.fractional over the whole access).
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;

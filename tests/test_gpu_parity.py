@@ -140,6 +140,76 @@ def test_group_id_probe_bit_exact(variant):
     assert bool(is_sentinel(out[int(offs[-1]):]).all())
 
 
+# sizes around the 16-row MMA step, the 64-row wgrad stage and the 128/256-row tiles, an
+# empty expert between live ones and at the end
+PROBE_SIZES = [3, 0, 130, 1, 257, 16, 63, 64, 65, 15, 17, 300, 0]
+
+
+def _probe_dy(sizes, N, tail):
+    """dY[r, :] = e(r) + 1 for every row of group e (small integers, exact in bf16), NaN in the
+    rows past the last offset; returns (dY, offs, rows)."""
+    offs = workloads.offsets_from_sizes(sizes)
+    rows = int(offs[-1]) + tail
+    grp = np.concatenate([np.full(sz, e, np.float32) for e, sz in enumerate(sizes)])
+    dY = torch.full((rows, N), float("nan"), dtype=torch.float32)
+    dY[: int(offs[-1])] = torch.from_numpy(grp + 1)[:, None]
+    return dY.to(torch.bfloat16), offs, rows
+
+
+def test_wgrad_group_id_probe_bit_exact(variant):
+    """A[:,0]=1 (other columns 0), dY rows of group e all equal to e+1: dW[e][0, n] is the
+    integer m_e (e+1), summed exactly in fp32 and rounded once to bf16, and every other dW
+    element is 0; a row counted in the wrong group, a row of the NaN tail read into a sum or
+    a lost tail row of a 64-row stage changes the bits."""
+    sizes = PROBE_SIZES
+    E, K, N = len(sizes), 136, 264
+    dY, offs, rows = _probe_dy(sizes, N, tail=40)
+    A = torch.zeros(rows, K, dtype=torch.bfloat16)
+    A[:, 0] = 1
+    A[int(offs[-1]):] = float("nan")
+    dW = sentinel((E, K, N))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    gg.wgrad(A.cuda(), dY.cuda(), torch.from_numpy(offs).cuda(), dW, status=st)
+    torch.cuda.synchronize()
+    s = int(st.item())
+    assert s & gg.DEV_LAUNCHED and (s & gg.DEV_ERROR_MASK) == 0
+    expect = torch.zeros(E, K, N, dtype=torch.float32)
+    for e, m in enumerate(sizes):
+        expect[e, 0, :] = float(m * (e + 1))
+    expect = expect.to(torch.bfloat16).cuda()   # one rounding of the exact integer
+    assert torch.equal(dW.view(torch.int16), expect.view(torch.int16))
+
+
+def test_dgrad_group_id_probe_bit_exact(variant):
+    """dY[:,0]=1 (other columns 0), W[e][:, 0]=e+1: dX[r, k] = e(r)+1 exactly for every row of
+    every group; the rows past the last offset keep their sentinel."""
+    sizes = PROBE_SIZES
+    E, K, N = len(sizes), 264, 72
+    offs = workloads.offsets_from_sizes(sizes)
+    rows = int(offs[-1]) + 24
+    dY = torch.zeros(rows, N, dtype=torch.bfloat16)
+    dY[:, 0] = 1
+    W = torch.zeros(E, K, N, dtype=torch.bfloat16)
+    for e in range(E):
+        W[e, :, 0] = e + 1
+    dX = sentinel((rows, K))
+    gg.dgrad(dY.cuda(), W.cuda(), torch.from_numpy(offs).cuda(), dX)
+    torch.cuda.synchronize()
+    grp = np.concatenate([np.full(sz, e) for e, sz in enumerate(sizes)])
+    expect = torch.from_numpy(grp + 1).float().cuda()[:, None].expand(-1, K)
+    assert bool((dX[: int(offs[-1])].float() == expect).all())
+    assert bool(is_sentinel(dX[int(offs[-1]):]).all())
+
+
+@pytest.mark.slow
+def test_gateup_config_full_elementwise():
+    """The E=64 Zipf gate-up config (K=2048, N=1536, 4 empty experts, unaligned sizes) in full:
+    every element of out, dX (all rows of every group) and dW against the oracle, with NaN
+    tail rows; the automatic launch shapes."""
+    r = workloads.make_ragged("gateup", tail=128, device="cuda")
+    check_ragged(r, sample=False)
+
+
 def test_masked_config_full():
     """Masked layout E=8, mmax=128, K=768, N=2048; NaN in inactive rows."""
     m = workloads.make_masked()
@@ -199,6 +269,63 @@ def test_masked_counts_across_box_and_tile_edges(N):
     ref, act, _ = oracle.masked_forward(m.A, m.W, m.masked_m)
     flat = out.view(-1, m.N)
     assert_close(to_f64(flat[torch.from_numpy(np.nonzero(act)[0]).cuda()]), ref[act], "masked")
+    assert bool(is_sentinel(flat[torch.from_numpy(np.nonzero(~act)[0]).cuda()]).all())
+
+
+@pytest.mark.parametrize("E,mmax,K,N,counts", [
+    (5, 40, 200, 136, [40, 0, 17, 1, 33]),        # mmax and K off the 32-row box / 64 grid
+    (3, 100, 776, 392, [100, 64, 99]),            # N without 64-wide chunks, 13 K blocks
+    (4, 300, 64, 128, [300, 129, 0, 257]),        # three 128-row blocks per expert
+    (70, 16, 128, 256, None),                     # many experts, 16-row capacity
+])
+def test_masked_forward_shapes(E, mmax, K, N, counts):
+    """Masked forward over shapes around the kernel's blocks: the active rows of each expert
+    in blocks of up to 128 (32-row boxes), 128-column weight tiles, 64-deep stages; inactive
+    rows NaN in A and untouched in out."""
+    if counts is None:
+        counts = np.random.default_rng(7).integers(0, mmax + 1, E)
+    m = workloads.make_masked(E=E, mmax=mmax, K=K, N=N, masked_m=counts, seed=63)
+    out = sentinel((E, mmax, N))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    gg.masked_forward(m.A.cuda(), m.W.cuda(), torch.from_numpy(m.masked_m).cuda(), out,
+                      status=st)
+    torch.cuda.synchronize()
+    s = int(st.item())
+    assert s & gg.DEV_LAUNCHED and (s & gg.DEV_ERROR_MASK) == 0
+    ref, act, _ = oracle.masked_forward(m.A, m.W, m.masked_m)
+    flat = out.view(-1, N)
+    assert_close(to_f64(flat[torch.from_numpy(np.nonzero(act)[0]).cuda()]), ref[act], "masked")
+    assert bool(is_sentinel(flat[torch.from_numpy(np.nonzero(~act)[0]).cuda()]).all())
+
+
+@pytest.mark.parametrize("with_scale", [False, True])
+def test_masked_forward_bias_scale(with_scale):
+    """Masked forward with the fused bias (and per-row bias scale, NaN in inactive rows so a
+    read of one would show): h = A W[e] + s[e*mmax + r] bias[e] for active rows only."""
+    m = workloads.make_masked(E=6, mmax=72, K=256, N=384, masked_m=[72, 0, 5, 33, 64, 1],
+                              seed=65)
+    g = torch.Generator().manual_seed(9)
+    bias = torch.randn(m.E, m.N, generator=g).to(torch.bfloat16)
+    scale = None
+    if with_scale:
+        scale = torch.randn(m.E * m.mmax, generator=g, dtype=torch.float32)
+        act_rows = np.zeros(m.E * m.mmax, bool)
+        for e in range(m.E):
+            act_rows[e * m.mmax: e * m.mmax + int(m.masked_m[e])] = True
+        scale[torch.from_numpy(~act_rows)] = float("nan")
+    out = sentinel((m.E, m.mmax, m.N))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    gg.masked_forward_ex(m.A.cuda(), m.W.cuda(), torch.from_numpy(m.masked_m).cuda(), out,
+                         bias=bias.cuda(), bias_scale=None if scale is None else scale.cuda(),
+                         status=st)
+    torch.cuda.synchronize()
+    s = int(st.item())
+    assert s & gg.DEV_LAUNCHED and (s & gg.DEV_ERROR_MASK) == 0
+    ref, act, _ = oracle.masked_forward_ex(m.A, m.W, m.masked_m, bias,
+                                           None if scale is None else scale.numpy(), 0)
+    flat = out.view(-1, m.N)
+    assert_close(to_f64(flat[torch.from_numpy(np.nonzero(act)[0]).cuda()]), ref[act],
+                 "masked bias")
     assert bool(is_sentinel(flat[torch.from_numpy(np.nonzero(~act)[0]).cuda()]).all())
 
 

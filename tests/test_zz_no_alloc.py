@@ -3,10 +3,11 @@ route (a runtime whose device memory is all reserved by its own allocator, or co
 not enter the CUDA allocator at that point). It takes no workspace: its histograms live in a
 fixed array inside the library, shared by every call.
 
-Checked through the C ABI against gg_route (which takes a caller-provided workspace): the
-offsets, packed rows and packed activations must be identical, on two calls in a row with
-different inputs (the shared array keeps the first call's contents). This file is collected
-last so that a run stopping at its first failure has run every other test already.
+Checked through the C ABI against gg_route (which takes a caller-provided workspace) and
+against the oracle's routing: the offsets, packed rows and packed activations must be
+identical, on two calls in a row with different inputs (the shared array keeps the first
+call's contents), and at the largest size the array admits. This file is collected last so
+that a run stopping at its first failure has run every other test already.
 """
 import ctypes
 
@@ -14,6 +15,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import workloads
 from conftest import cuda_ok
 
@@ -60,6 +62,14 @@ def test_route_noalloc_matches_route_on_two_calls_in_a_row():
         total = int(ref_offs[-1].item())
         # integer and copy work: bit-exact
         assert torch.equal(A[:total].view(torch.int16), ref_A[:total].view(torch.int16))
+        _check_against_oracle(ids_np, X, E, A, row_of, offs)
+
+
+def _check_against_oracle(ids_np, X, E, A, row_of, offs):
+    roffs, rrow, rA, _ = oracle.route(ids_np, X.cpu(), E)
+    np.testing.assert_array_equal(offs.cpu().numpy(), roffs)
+    np.testing.assert_array_equal(row_of.cpu().numpy(), rrow)
+    np.testing.assert_array_equal(oracle.as_u16(A[: int(roffs[-1])]), rA)
 
 
 def test_route_noalloc_rejects_problems_beyond_its_array():
@@ -73,10 +83,21 @@ def test_route_noalloc_rejects_problems_beyond_its_array():
     rc = _noalloc_fn()(ids.data_ptr(), T, k, E, X.data_ptr(), 8, A.data_ptr(), row_of.data_ptr(),
                        offs.data_ptr(), None, torch.cuda.current_stream().cuda_stream)
     assert rc == 4 and "TOO_LARGE" in gg.status_string(rc)
-    # the largest allowed size with 1024 experts is accepted
-    T = 16384
-    rc = _noalloc_fn()(ids.data_ptr(), T, k, E, X.data_ptr(), 8, A.data_ptr(), row_of.data_ptr(),
-                       offs.data_ptr(), None, torch.cuda.current_stream().cuda_stream)
+
+
+def test_route_noalloc_at_the_largest_size_of_its_array():
+    """T=16384 tokens x top-4 over 1024 experts fills all GG_ROUTE_NOALLOC_MAX_COUNTS entries
+    (256 blocks x 1024 experts): varied expert ids, so that a wrong bound or histogram index at
+    the array's end would show in the offsets, the packed rows or the packed activations."""
+    T, k, E, K = 16384, 4, 1024, 8
+    ids_np, X = workloads.make_routing(T, k, E, K, seed=131, dropped=17)
+    ids, X = torch.from_numpy(ids_np).cuda(), X.cuda()
+    A, row_of, offs, st = _route_noalloc(ids, X, E)
+    ref_A, ref_row, ref_offs = gg.route(ids, X, E)
     torch.cuda.synchronize()
-    assert rc == 0
-    assert int(offs[0].item()) == T * k
+    assert (int(st.item()) & gg.DEV_ERROR_MASK) == 0
+    assert torch.equal(offs, ref_offs)
+    assert torch.equal(row_of, ref_row)
+    total = int(ref_offs[-1].item())
+    assert torch.equal(A[:total].view(torch.int16), ref_A[:total].view(torch.int16))
+    _check_against_oracle(ids_np, X, E, A, row_of, offs)
