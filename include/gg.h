@@ -187,14 +187,19 @@ GG_API gg_status gg_masked_forward(const void* A, const void* W, const int32_t* 
  *   GG_FLAG_W_NK       W (and dW) stored [E, N, K]: each expert's weight out-major, the way
  *                      TransformerEngine's GroupedLinear keeps it (TransformerEngine PR 3542,
  *                      "Changes": dispatch of the transposed operand layouts); forward
- *                      computes A . W[e]^T */
+ *                      computes A . W[e]^T
+ *   GG_FLAG_GATE_UP_CONCAT  with GG_ACT_SILU_MUL only (else GG_ERR_INVALID_ARG): gate and up
+ *                      are the two halves of W's N columns, [gate | up], the usual layout of
+ *                      a fused gate-up weight: out[r, j] = silu(h[r, j]) * h[r, N/2 + j]
+ *                      (N % 256 == 0); accepted by gg_forward_ex and gg_masked_forward_ex */
 #define GG_FLAG_ZERO_TAIL 0x1
 #define GG_FLAG_W_NK 0x2
+#define GG_FLAG_GATE_UP_CONCAT 0x4
 typedef struct gg_epilogue {
   const void* bias;
   const float* bias_scale;
   int32_t act;
-  int32_t flags; /* GG_FLAG_ZERO_TAIL | GG_FLAG_W_NK */
+  int32_t flags; /* GG_FLAG_ZERO_TAIL | GG_FLAG_W_NK | GG_FLAG_GATE_UP_CONCAT */
 } gg_epilogue;
 
 /* gg_forward with a fused epilogue and flags (epi may be NULL: same as gg_forward). out is

@@ -33,7 +33,7 @@ MAX_EXPERTS = 1024
 _lib = None
 
 ACT_NONE, ACT_SILU_MUL = 0, 1
-FLAG_ZERO_TAIL, FLAG_W_NK = 0x1, 0x2
+FLAG_ZERO_TAIL, FLAG_W_NK, FLAG_GATE_UP_CONCAT = 0x1, 0x2, 0x4
 
 
 class _Epilogue(ctypes.Structure):
@@ -208,11 +208,13 @@ def _epilogue(bias, bias_scale, act, E, N, flags=0):
 def forward_ex(A: torch.Tensor, W: torch.Tensor, offs: torch.Tensor, out: torch.Tensor, *,
                bias: Optional[torch.Tensor] = None, bias_scale: Optional[torch.Tensor] = None,
                act: int = ACT_NONE, zero_tail: bool = False, w_nk: bool = False,
-               status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+               gate_up_concat: bool = False, status: Optional[torch.Tensor] = None,
+               stream=None) -> torch.Tensor:
     """Forward with a fused epilogue: h = A @ W[e] + bias_scale[r] * bias[e]; with
     act=ACT_SILU_MUL out = silu(gate) * up over gate/up column blocks of 128 (N % 256 == 0),
-    and out has N/2 columns. bias_scale is read only for rows inside a group. zero_tail
-    writes zeros to the rows past the last offset; w_nk takes W as [E, N, K]."""
+    or, with gate_up_concat, over the two halves [gate | up] of W's columns; out has N/2
+    columns. bias_scale is read only for rows inside a group. zero_tail writes zeros to the
+    rows past the last offset; w_nk takes W as [E, N, K]."""
     _check(A, "A", torch.bfloat16, 2)
     _check(W, "W", torch.bfloat16, 3)
     _check(offs, "offs", torch.int32, 1)
@@ -225,7 +227,8 @@ def forward_ex(A: torch.Tensor, W: torch.Tensor, offs: torch.Tensor, out: torch.
     ncols = N // 2 if act == ACT_SILU_MUL else N
     if K2 != K or offs.numel() != E or tuple(out.shape) != (rows, ncols):
         raise ValueError("shape mismatch: A[rows,K], W[E,K,N], offs[E], out[rows,N or N/2]")
-    epi = _epilogue(bias, bias_scale, act, E, N, _flags(zero_tail, w_nk))
+    flags = _flags(zero_tail, w_nk) | (FLAG_GATE_UP_CONCAT if gate_up_concat else 0)
+    epi = _epilogue(bias, bias_scale, act, E, N, flags)
     rc = lib().gg_forward_ex(_ptr(A), _ptr(W), _ptr(offs), _ptr(out), rows, K, N, E,
                              ctypes.byref(epi), _status_ptr(status), _stream_handle(stream))
     _raise(rc, "gg_forward_ex")
@@ -277,7 +280,8 @@ def wgrad_ex(A: torch.Tensor, dY: torch.Tensor, offs: torch.Tensor, dW: torch.Te
 def masked_forward_ex(A: torch.Tensor, W: torch.Tensor, masked_m: torch.Tensor,
                       out: torch.Tensor, *, bias: Optional[torch.Tensor] = None,
                       bias_scale: Optional[torch.Tensor] = None, act: int = ACT_NONE,
-                      status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                      gate_up_concat: bool = False, status: Optional[torch.Tensor] = None,
+                      stream=None) -> torch.Tensor:
     """Masked forward with the fused epilogue of forward_ex; bias_scale is indexed by the
     flat row e*mmax + r; out is [E, mmax, N] or [E, mmax, N/2]."""
     _check(A, "A", torch.bfloat16, 3)
@@ -289,7 +293,8 @@ def masked_forward_ex(A: torch.Tensor, W: torch.Tensor, masked_m: torch.Tensor,
     ncols = N // 2 if act == ACT_SILU_MUL else N
     if E2 != E or K2 != K or masked_m.numel() != E or tuple(out.shape) != (E, mmax, ncols):
         raise ValueError("shape mismatch: A[E,mmax,K], W[E,K,N], masked_m[E], out")
-    epi = _epilogue(bias, bias_scale, act, E, N)
+    epi = _epilogue(bias, bias_scale, act, E, N,
+                    FLAG_GATE_UP_CONCAT if gate_up_concat else 0)
     rc = lib().gg_masked_forward_ex(_ptr(A), _ptr(W), _ptr(masked_m), _ptr(out), mmax, K, N, E,
                                     ctypes.byref(epi), _status_ptr(status),
                                     _stream_handle(stream))
@@ -510,7 +515,7 @@ def grouped_mm(A: torch.Tensor, W: torch.Tensor, offs: torch.Tensor,
 
 __all__ = [
     "forward", "forward_ex", "dgrad", "dgrad_ex", "wgrad", "wgrad_ex", "wgrad_f32",
-    "masked_forward", "FLAG_ZERO_TAIL", "FLAG_W_NK",
+    "masked_forward", "FLAG_ZERO_TAIL", "FLAG_W_NK", "FLAG_GATE_UP_CONCAT",
     "masked_forward_ex", "ACT_NONE", "ACT_SILU_MUL", "route", "route_workspace_bytes",
     "grouped_mm", "layer_step_host", "status_string", "version",
     "set_watchdog_ns", "testing_skip_first_load", "testing_force_variant", "lib", "GGError",

@@ -466,8 +466,11 @@ gg_status set_epilogue(gg::Params* p, const gg_epilogue* epi, int64_t N) {
   if (epi->bias_scale != nullptr && (reinterpret_cast<uintptr_t>(epi->bias_scale) & 3u) != 0)
     return GG_ERR_UNSUPPORTED;
   if (epi->act == GG_ACT_SILU_MUL && (N % kBN) != 0) return GG_ERR_UNSUPPORTED;
+  if ((epi->flags & GG_FLAG_GATE_UP_CONCAT) && epi->act != GG_ACT_SILU_MUL)
+    return GG_ERR_INVALID_ARG;
   p->bias = reinterpret_cast<const __nv_bfloat16*>(epi->bias);
   p->bias_scale = epi->bias != nullptr ? epi->bias_scale : nullptr;
+  p->gate_up_concat = (epi->flags & GG_FLAG_GATE_UP_CONCAT) ? 1 : 0;
   return GG_OK;
 }
 
@@ -484,19 +487,23 @@ gg_status forward_impl(const void* A, const void* W, const int32_t* offs, void* 
   if (A == nullptr || out == nullptr) return GG_ERR_INVALID_ARG;
   if (!aligned16(A) || !aligned16(W) || !aligned16(out)) return GG_ERR_UNSUPPORTED;
   const int32_t flags = epi != nullptr ? epi->flags : 0;
-  if (flags & ~(GG_FLAG_ZERO_TAIL | GG_FLAG_W_NK)) return GG_ERR_INVALID_ARG;
+  if (flags & ~(GG_FLAG_ZERO_TAIL | GG_FLAG_W_NK | GG_FLAG_GATE_UP_CONCAT))
+    return GG_ERR_INVALID_ARG;
   const bool silu = epi != nullptr && epi->act == GG_ACT_SILU_MUL;
   const bool wnk = (flags & GG_FLAG_W_NK) != 0;
+  // [gate | up] weights are loaded as 128-column gate and up blocks
+  const bool concat = (flags & GG_FLAG_GATE_UP_CONCAT) != 0;
   const bool pair = use_pair(rows_alloc, E);
   const bool wide = pair && use_wide(rows_alloc, E, K);
   const bool chunked = (N % 64) == 0;
   const uint32_t bcols = wide ? kWideBN / 2 : pair ? kBN / 2 : kBN;
+  const uint32_t bbox = concat ? 128u : bcols;  // columns of W per box
   CUtensorMap ma, mb;
   if (!map_2d(&ma, A, rows_alloc, K, 64, gg::BM)) return GG_ERR_CUDA;
   if (wnk) {
     // W[e] is [N, K]: K-major B, one box of bcols rows of N per stage
-    if (!map_w(&mb, W, E, N, K, 64, bcols)) return GG_ERR_CUDA;
-  } else if (chunked ? !map_w_chunked(&mb, W, E, K, N, 64, bcols / 64)
+    if (!map_w(&mb, W, E, N, K, 64, bbox)) return GG_ERR_CUDA;
+  } else if (chunked ? !map_w_chunked(&mb, W, E, K, N, 64, bbox / 64)
                      : !map_w(&mb, W, E, K, N, 64, 64)) {
     return GG_ERR_CUDA;
   }
@@ -682,6 +689,7 @@ gg_status masked_impl(const void* A, const void* W, const int32_t* masked_m, voi
   gg_status s = check_common((int64_t)E * mmax, K, N, E, masked_m, dev_status, &di);
   if (s != GG_OK) return s;
   if (W == nullptr) return GG_ERR_INVALID_ARG;
+  if (epi != nullptr && (epi->flags & ~GG_FLAG_GATE_UP_CONCAT)) return GG_ERR_INVALID_ARG;
   if (mmax == 0) return GG_OK;
   if (A == nullptr || out == nullptr) return GG_ERR_INVALID_ARG;
   if (!aligned16(A) || !aligned16(W) || !aligned16(out)) return GG_ERR_UNSUPPORTED;
@@ -695,7 +703,9 @@ gg_status masked_impl(const void* A, const void* W, const int32_t* masked_m, voi
   const bool chunked = (N % 64) == 0;
   CUtensorMap ma, mb;
   if (!map_2d(&ma, A, (int64_t)E * mmax, K, 64, 32)) return GG_ERR_CUDA;
-  if (chunked ? !map_w_chunked(&mb, W, E, K, N, 64, bn / 64) : !map_w(&mb, W, E, K, N, 64, 64))
+  const bool concat = (epi->flags & GG_FLAG_GATE_UP_CONCAT) != 0;  // 128-column blocks
+  if (chunked ? !map_w_chunked(&mb, W, E, K, N, 64, (concat ? 128 : bn) / 64)
+              : !map_w(&mb, W, E, K, N, 64, 64))
     return GG_ERR_CUDA;
   gg::Params p = base_params(masked_m, out, dev_status, (int64_t)E * mmax, E);
   p.b_chunked = chunked ? 1 : 0;

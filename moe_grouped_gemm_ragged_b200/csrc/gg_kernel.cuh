@@ -137,6 +137,10 @@ struct Params {
   // forward/dgrad: rows at and past the last effective offset are written with zeros (a
   // pseudo-group after the last expert whose tiles have no reduction stages)
   int32_t zero_tail;
+  // SiLU-and-mul with W's columns as [gate | up] halves (0: gate and up interleaved in
+  // blocks of 128); the loads put the tile's gate block and up block side by side, so the
+  // accumulator holds the same columns in both layouts
+  int32_t gate_up_concat;
 };
 
 template <int BN, int STAGES, bool PAIR, int BKL = BK>
@@ -574,7 +578,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint32_t fb_leader = ptx::mapa(ptx::smem_u32(fb), 0);
             if (leader) ptx::mbar_arrive_expect_tx(fb, 2 * L::STAGE_BYTES);
             ptx::tma_load_2d_pair(sA, &mapA, fb_leader, kb * BKM, tl.a_row0 + row_off, pol_tok);
-            if constexpr (MODE == Mode::Dgrad) {
+            if (ACT == 1 && p.gate_up_concat) {
+              // [gate | up] weights: this CTA's B columns are 128-wide gate and up blocks
+              // (a 256-wide pair tile: the leader's gate block, the follower's up block)
+              constexpr int PIECES = L::B_COLS / 128;
+              for (int i = 0; i < PIECES; ++i) {
+                const int32_t gu = PIECES == 1 ? (int32_t)rank : i;
+                const int32_t blk = PIECES == 1 ? 0 : (int32_t)rank;
+                const int32_t col = gu * (p.prod_cols / 2) + tl.n0 / 2 + 128 * blk;
+                uint8_t* dst = sB + i * (128 * BKM * 2);
+                if constexpr (MODE == Mode::Dgrad)
+                  ptx::tma_load_3d_pair(dst, &mapB, fb_leader, kb * BKM, col, tl.e, pol_w);
+                else
+                  ptx::tma_load_4d_pair(dst, &mapB, fb_leader, 0, kb * BKM, col / 64, tl.e, pol_w);
+              }
+            } else if constexpr (MODE == Mode::Dgrad) {
               ptx::tma_load_3d_pair(sB, &mapB, fb_leader, kb * BKM, tl.n0 + col_off, tl.e, pol_w);
             } else if (p.b_chunked) {
               ptx::tma_load_4d_pair(sB, &mapB, fb_leader, 0, kb * BKM, (tl.n0 + col_off) / 64,
@@ -607,7 +625,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if constexpr (MODE == Mode::Forward || MODE == Mode::Masked) {
               if constexpr (MODE == Mode::Forward)
                 ptx::tma_load_2d(sA, &mapA, lb, kb * BKM, tl.a_row0, pol_tok);
-              if (p.b_chunked) {
+              if (ACT == 1 && p.gate_up_concat) {
+                // [gate | up] weights: the tile's gate block, then its up block
+                for (int i = 0; i < 2; ++i)
+                  ptx::tma_load_4d(sB + i * (128 * BKM * 2), &mapB, lb, 0, kb * BKM,
+                                   (i * (p.prod_cols / 2) + tl.n0 / 2) / 64, tl.e, pol_w);
+              } else if (p.b_chunked) {
                 ptx::tma_load_4d(sB, &mapB, lb, 0, kb * BKM, tl.n0 / 64, tl.e, pol_w);
               } else {
 #pragma unroll
@@ -616,7 +639,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               }
             } else if constexpr (MODE == Mode::Dgrad) {
               ptx::tma_load_2d(sA, &mapA, lb, kb * BKM, tl.a_row0, pol_tok);
-              ptx::tma_load_3d(sB, &mapB, lb, kb * BKM, tl.n0, tl.e, pol_w);
+              if (ACT == 1 && p.gate_up_concat) {
+                for (int i = 0; i < 2; ++i)
+                  ptx::tma_load_3d(sB + i * (128 * BKM * 2), &mapB, lb, kb * BKM,
+                                   i * (p.prod_cols / 2) + tl.n0 / 2, tl.e, pol_w);
+              } else {
+                ptx::tma_load_3d(sB, &mapB, lb, kb * BKM, tl.n0, tl.e, pol_w);
+              }
             } else {  // Wgrad
               const int32_t r = tl.tok0 + kb * BKM;
               if (p.a_chunked) {
@@ -872,9 +901,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
                 const int32_t t = half + c + 8 * j;
-                const int32_t gcol = tl.n0 + 256 * (t / 128) + t % 128;
+                // gate and up columns of output column n0/2 + t
+                const int32_t gcol = p.gate_up_concat ? tl.n0 / 2 + t
+                                                      : tl.n0 + 256 * (t / 128) + t % 128;
+                const int32_t ucol = p.gate_up_concat ? gcol + p.prod_cols / 2 : gcol + 128;
                 const uint4 bg = __ldg(reinterpret_cast<const uint4*>(bias_e + gcol));
-                const uint4 bu = __ldg(reinterpret_cast<const uint4*>(bias_e + gcol + 128));
+                const uint4 bu = __ldg(reinterpret_cast<const uint4*>(bias_e + ucol));
                 const __nv_bfloat16* g8 = reinterpret_cast<const __nv_bfloat16*>(&bg);
                 const __nv_bfloat16* u8 = reinterpret_cast<const __nv_bfloat16*>(&bu);
 #pragma unroll

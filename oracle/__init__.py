@@ -172,13 +172,15 @@ def wgrad_accumulate(A, dY, offs, old, alpha: float, beta: float, ks=None, threa
     return out
 
 
-def epilogue(h, groups, rows, bias=None, bias_scale=None, act: int = 0):
+def epilogue(h, groups, rows, bias=None, bias_scale=None, act: int = 0, concat: bool = False):
     """The forward epilogue on fp64 products h[nrows, N] of rows ``rows`` whose groups are
     ``groups`` (rows in no group stay NaN):
       h'[r, n] = h[r, n] + s[r] * bias[e(r), n]      (s = bias_scale, 1 when absent)
-    act 0: h'; act 1 (SiLU-and-mul, gate/up interleaved in blocks of 128 columns):
+    act 0: h'; act 1 (SiLU-and-mul), gate/up interleaved in blocks of 128 columns:
       out[r, 128 b + i] = silu(h'[r, 256 b + i]) * h'[r, 256 b + 128 + i],
-      silu(x) = x / (1 + exp(-x))
+    or, with concat, gate and up as the two halves of the N columns:
+      out[r, j] = silu(h'[r, j]) * h'[r, N/2 + j],
+    silu(x) = x / (1 + exp(-x))
     (TransformerEngine PR 3542 review: per-group bias and a per-token bias scale over the
     logical rows; sglang PR 32385, "Cause": SiLU-and-mul between the gate-up and down GEMMs)."""
     h = np.array(h, dtype=np.float64, copy=True)
@@ -192,6 +194,9 @@ def epilogue(h, groups, rows, bias=None, bias_scale=None, act: int = 0):
         return h
     N = h.shape[1]
     assert N % 256 == 0
+    if concat:
+        gate, up = h[:, : N // 2], h[:, N // 2:]
+        return gate / (1.0 + np.exp(-gate)) * up
     nb = N // 256
     hv = h.reshape(len(h), nb, 2, 128)
     gate, up = hv[:, :, 0, :], hv[:, :, 1, :]
@@ -199,22 +204,23 @@ def epilogue(h, groups, rows, bias=None, bias_scale=None, act: int = 0):
     return out.reshape(len(h), N // 2)
 
 
-def forward_ex(A, W, offs, bias=None, bias_scale=None, act: int = 0, rows=None, threads=None):
+def forward_ex(A, W, offs, bias=None, bias_scale=None, act: int = 0, rows=None, threads=None,
+               concat: bool = False):
     """Forward with the epilogue above. Returns (out[nrows, N or N/2], group_of[nrows])."""
     h, g = forward(A, W, offs, rows=rows, threads=threads)
     r = np.arange(h.shape[0]) if rows is None else np.asarray(rows, np.int64)
-    return epilogue(h, g, r, bias, bias_scale, act), g
+    return epilogue(h, g, r, bias, bias_scale, act, concat), g
 
 
 def masked_forward_ex(A, W, masked_m, bias=None, bias_scale=None, act: int = 0, rows=None,
-                      threads=None):
+                      threads=None, concat: bool = False):
     """Masked forward with the epilogue above; bias_scale is indexed by flat row e*mmax+r.
     Returns (out, active, bad)."""
     h, act_rows, bad = masked_forward(A, W, masked_m, rows=rows, threads=threads)
     E, mmax, _ = as_u16(A).shape
     r = np.arange(E * mmax) if rows is None else np.asarray(rows, np.int64)
     g = np.where(act_rows, r // mmax, -1)
-    return epilogue(h, g, r, bias, bias_scale, act), act_rows, bad
+    return epilogue(h, g, r, bias, bias_scale, act, concat), act_rows, bad
 
 
 def route(topk_ids, X, E: int):

@@ -395,6 +395,46 @@ def test_forward_epilogue_bias_scale_silu(act, with_bias, with_scale, variant):
     assert bool(is_sentinel(out[T:]).all())
 
 
+@pytest.mark.parametrize("with_bias,w_nk", [(False, False), (True, False), (True, True)])
+def test_forward_silu_mul_concatenated_gate_up(with_bias, w_nk, variant):
+    """SiLU-and-mul with W's columns as [gate | up] (GG_FLAG_GATE_UP_CONCAT): out[r, j] =
+    silu(h[r, j]) * h[r, N/2 + j] against the oracle's concatenated reading, on every launch
+    shape and with W stored [E, N, K]; rows past the last offset keep their sentinel."""
+    sizes = [0, 1, 127, 128, 129, 300, 17, 600]
+    K, N = 192, 1024
+    r = workloads.make_ragged_custom(len(sizes), K, N, sizes, seed=85, tail=40)
+    A, W = r.A.cuda(), r.W.cuda()
+    offs = torch.from_numpy(r.offs).cuda()
+    g = torch.Generator().manual_seed(6)
+    bias = torch.randn(r.E, N, generator=g).to(torch.bfloat16) if with_bias else None
+    Wk = W.transpose(1, 2).contiguous() if w_nk else W
+    out = sentinel((r.rows_alloc, N // 2))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    gg.forward_ex(A, Wk, offs, out, bias=None if bias is None else bias.cuda(),
+                  act=gg.ACT_SILU_MUL, gate_up_concat=True, w_nk=w_nk, status=st)
+    torch.cuda.synchronize()
+    s = int(st.item())
+    assert s & gg.DEV_LAUNCHED and (s & gg.DEV_ERROR_MASK) == 0
+    ref, _ = oracle.forward_ex(r.A, r.W, r.offs, bias, None, 1, concat=True)
+    assert_close(to_f64(out[: r.T]), ref[: r.T], "forward silu concat")
+    assert bool(is_sentinel(out[r.T:]).all())
+
+
+def test_masked_forward_silu_mul_concatenated_gate_up():
+    """The masked gate-up GEMM with fused SiLU-and-mul over [gate | up] weight halves."""
+    m = workloads.make_masked(E=8, mmax=128, K=768, N=1536, seed=87)
+    bias = torch.randn(8, 1536).to(torch.bfloat16)
+    out = sentinel((8, 128, 768))
+    gg.masked_forward_ex(m.A.cuda(), m.W.cuda(), torch.from_numpy(m.masked_m).cuda(), out,
+                         bias=bias.cuda(), act=gg.ACT_SILU_MUL, gate_up_concat=True)
+    torch.cuda.synchronize()
+    ref, act, _ = oracle.masked_forward_ex(m.A, m.W, m.masked_m, bias, None, 1, concat=True)
+    flat = out.view(-1, 768)
+    assert_close(to_f64(flat[torch.from_numpy(np.nonzero(act)[0]).cuda()]), ref[act],
+                 "masked silu concat")
+    assert bool(is_sentinel(flat[torch.from_numpy(np.nonzero(~act)[0]).cuda()]).all())
+
+
 def test_masked_forward_silu_mul_on_the_sglang_shape():
     """The masked down-GEMM input: gate-up GEMM of the masked layout with fused SiLU-and-mul,
     written only for the active rows (inactive rows NaN in A, sentinel in out)."""

@@ -2,6 +2,8 @@
 regions around outputs, CUDA-graph capture with offsets changed between replays, a
 concurrent copy stream, and the in-kernel watchdog (a wait that runs out returns a status;
 no GPU fault, trap or hang is involved)."""
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -105,6 +107,19 @@ def test_host_rejections_with_device_buffers():
     with pytest.raises(gg.GGError):
         gg.forward(A[:, :60].contiguous(), W[:, :60].contiguous(), offs,
                    torch.zeros(64, 64, dtype=torch.bfloat16, device=dev))
+    # the [gate | up] flag without the SiLU-and-mul epilogue, and a flag the masked call
+    # does not take, are rejected before any launch
+    with pytest.raises(gg.GGError) as ei:
+        gg.forward_ex(A, W, offs, out, gate_up_concat=True)
+    assert ei.value.code == gg.GG_ERR_INVALID_ARG
+    with pytest.raises(gg.GGError) as ei:
+        gg.masked_forward_ex(A.view(2, 32, 64), W, offs, out.view(2, 32, 64),
+                             gate_up_concat=True)
+    assert ei.value.code == gg.GG_ERR_INVALID_ARG
+    epi = gg._Epilogue(None, None, gg.ACT_NONE, gg.FLAG_ZERO_TAIL)
+    assert L.gg_masked_forward_ex(A.data_ptr(), W.data_ptr(), offs.data_ptr(), out.data_ptr(),
+                                  32, 64, 64, 2, ctypes.byref(epi), None,
+                                  stream) == gg.GG_ERR_INVALID_ARG
     torch.cuda.synchronize()
 
 

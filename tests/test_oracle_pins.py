@@ -369,6 +369,34 @@ def test_epilogue_silu_mul_layout_and_closed_form():
             assert abs(out[3, 128 * b + i] - want) <= 1e-15 * max(1.0, abs(want))
 
 
+def test_epilogue_silu_mul_concatenated_halves():
+    """The same exact labels with gate and up as the two halves of N: output column j must be
+    silu(gate column j) * up column N/2 + j; and permuting W's columns from the concatenated
+    order into the 128-block interleaved order gives the interleaved result bit for bit."""
+    import math
+    N, K = 512, 16
+    A = torch.zeros(4, K, dtype=torch.bfloat16)
+    A[:, 0] = 1
+    n = torch.arange(N, dtype=torch.float32)
+    labels = torch.where(n < 256, n / 64.0, (n - 384.0) / 64.0)  # <= 8 significant bits
+    W = torch.zeros(1, K, N, dtype=torch.bfloat16)
+    W[0, 0, :] = labels
+    out, _ = oracle.forward_ex(A, W, [4], act=1, concat=True)
+    assert out.shape == (4, N // 2)
+    for j in range(N // 2):
+        gte, up = float(labels[j]), float(labels[N // 2 + j])
+        want = gte / (1.0 + math.exp(-gte)) * up
+        assert abs(out[3, j] - want) <= 1e-15 * max(1.0, abs(want))
+    # concatenated column c -> interleaved position: gate j -> 256 (j // 128) + j % 128,
+    # up j -> that + 128
+    perm = torch.empty(N, dtype=torch.long)
+    j = torch.arange(N // 2)
+    perm[256 * (j // 128) + j % 128] = j
+    perm[256 * (j // 128) + 128 + j % 128] = N // 2 + j
+    inter, _ = oracle.forward_ex(A, W[:, :, perm], [4], act=1)
+    np.testing.assert_array_equal(inter, out)
+
+
 def _route_brute(ids, X, E):
     """Obviously-correct routing: for each expert in order, every assignment in order."""
     ids = np.asarray(ids)
