@@ -40,8 +40,12 @@ UNIT = "TFLOP/s"
 # capture of ONE launch of ONE kernel (-k <kernel> -c 1) with only these counters, which ncu
 # collects in a single pass; a launch list over many kernels collects gpu__time_duration.sum
 # alone.
-NCU_TRAFFIC = {}
-NCU_TRAFFIC_SRC_HASH = ""
+NCU_TRAFFIC = {
+    ("forward", "large"): 11.103e9,
+    ("dgrad", "large"): 12.583e9,
+    ("wgrad", "large"): 19.867e9,
+}
+NCU_TRAFFIC_SRC_HASH = "5794e31d918ee2ec"
 
 
 GEMM_SOURCES = ("gg_kernel.cuh", "ptx.cuh", "gg_api.cu", "gg_masked.cuh")  # kernels + launch
@@ -786,6 +790,58 @@ def run_table(args):
     return 0
 
 
+def run_launch_only(args):
+    """Launch the chosen passes of one workload `--reps` times each, in order, untimed: the
+    command that `ncu` captures (select the launch with -k / -s / -c). Workloads: the ragged
+    configs of --workload, or "tiny" (4 experts, offsets (8,16,32,40)), "masked" (the
+    sglang shape) and "route" (the token routing of the large shape's rows: 32768 tokens,
+    top-8 of 16 experts, K=6144; pass "route")."""
+    import workloads
+    import moe_grouped_gemm_ragged_b200 as gg
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (there is no CPU implementation)")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    passes = args.passes.split(",")
+    if args.workload == "masked":
+        m = workloads.make_masked(device=dev)
+        mm = torch.from_numpy(m.masked_m).to(dev)
+        mout = torch.empty((m.E, m.mmax, m.N), dtype=torch.bfloat16, device=dev)
+        fns = {"masked": lambda: gg.masked_forward(m.A, m.W, mm, mout)}
+    elif args.workload == "route":
+        tok, k, E, K = 32768, 8, 16, 6144
+        ids_np, X = workloads.make_routing(tok, k, E, K, seed=12, device=dev)
+        ids = torch.from_numpy(ids_np).to(dev)
+        a_packed = torch.empty((tok * k, K), dtype=torch.bfloat16, device=dev)
+        row_of = torch.empty(tok * k, dtype=torch.int32, device=dev)
+        roffs = torch.empty(E, dtype=torch.int32, device=dev)
+        wsp = torch.empty(max(4, gg.route_workspace_bytes(tok * k, E)), dtype=torch.uint8,
+                          device=dev)
+        fns = {"route": lambda: gg.route(ids, X, E, A_packed=a_packed, row_of=row_of,
+                                         offs=roffs, workspace=wsp)}
+    else:
+        r = (workloads.make_tiny((8, 16, 32, 40)) if args.workload == "tiny"
+             else workloads.make_ragged(args.workload, tail=0, device=dev))
+        A, W, dY = (t.to(dev) for t in (r.A, r.W, r.dY))
+        offs = torch.from_numpy(np.ascontiguousarray(r.offs)).to(dev)
+        out = torch.empty((r.rows_alloc, r.N), dtype=torch.bfloat16, device=dev)
+        dX = torch.empty((r.rows_alloc, r.K), dtype=torch.bfloat16, device=dev)
+        dW = torch.empty((r.E, r.K, r.N), dtype=torch.bfloat16, device=dev)
+        fns = {"forward": lambda: gg.forward(A, W, offs, out),
+               "dgrad": lambda: gg.dgrad(dY, W, offs, dX),
+               "wgrad": lambda: gg.wgrad(A, dY, offs, dW)}
+    for p in passes:
+        if p not in fns:
+            raise SystemExit(f"pass {p!r} is not one of {sorted(fns)} for {args.workload}")
+    torch.cuda.synchronize()
+    for _ in range(args.reps):
+        for p in passes:
+            fns[p]()
+    torch.cuda.synchronize()
+    print(f"launched {args.reps} x {passes} on {args.workload}", flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -793,7 +849,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="large",
-                    choices=["large", "large_unaligned", "gateup", "downproj", "large_e2"])
+                    choices=["large", "large_unaligned", "gateup", "downproj", "large_e2",
+                             "tiny", "masked", "route"],
+                    help="tiny, masked and route: with --launch-only")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--e2e-chunks", type=int, default=0,
                     help="expert chunks of the host-buffer pass (0: the library default)")
@@ -804,7 +862,16 @@ def main(argv=None):
                     help="launch shapes: 0 automatic, 1 single CTA, 2 CTA pair, 3 CTA pair with 256 x 512 wgrad tiles")
     ap.add_argument("--table", action="store_true",
                     help="per-config, per-pass table of every parity config (JSON lines)")
+    ap.add_argument("--launch-only", action="store_true",
+                    help="launch --passes of --workload --reps times, untimed (for ncu)")
+    ap.add_argument("--passes", default="forward,dgrad,wgrad",
+                    help="with --launch-only: forward, dgrad, wgrad (ragged) or masked")
+    ap.add_argument("--reps", type=int, default=2, help="with --launch-only")
     args = ap.parse_args(argv)
+    if args.launch_only:
+        return run_launch_only(args)
+    if args.workload in ("tiny", "masked", "route"):
+        ap.error("--workload tiny/masked/route needs --launch-only")
     if args.table:
         return run_table(args)
     if args.warmup < 3:
