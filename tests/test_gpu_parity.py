@@ -202,6 +202,45 @@ def test_dgrad_group_id_probe_bit_exact(variant):
 
 
 @pytest.mark.slow
+@pytest.mark.parametrize("name", ["large", "large_unaligned"])
+def test_large_group_id_probes_bit_exact(name):
+    """Group-id probes at the full size of the large shape (E=16, 262144 rows, K=6144,
+    N=4096), where the tolerance alone would not see one misassigned row: with A[:,0]=1 (other
+    columns 0) and W[e][0,:]=e+1, every element of out is e(r)+1; with dY rows of group e all
+    e+1, dW[e][0,n] is m_e (e+1), an exact fp32 sum rounded once to bf16, and every other dW
+    element is 0. Compared in full on the GPU; the automatic launch shapes."""
+    sizes = workloads.group_sizes(name)
+    E, K, N = len(sizes), 6144, 4096
+    offs = workloads.offsets_from_sizes(sizes)
+    T = int(offs[-1])
+    offs_d = torch.from_numpy(offs).cuda()
+    grp = torch.repeat_interleave(torch.arange(E, device="cuda"),
+                                  torch.from_numpy(np.asarray(sizes)).cuda())
+    A = torch.zeros(T, K, dtype=torch.bfloat16, device="cuda")
+    A[:, 0] = 1
+    W = torch.zeros(E, K, N, dtype=torch.bfloat16, device="cuda")
+    W[:, 0, :] = (torch.arange(E, device="cuda", dtype=torch.float32) + 1)[:, None].to(
+        torch.bfloat16)
+    out = torch.empty(T, N, dtype=torch.bfloat16, device="cuda")
+    st = torch.zeros(2, dtype=torch.int32, device="cuda")
+    gg.forward(A, W, offs_d, out, status=st[0:1])
+    del W
+    expect_row = (grp + 1).to(torch.bfloat16)
+    assert bool((out == expect_row[:, None]).all()), "forward: a row left its group"
+    del out
+    dY = expect_row[:, None].expand(T, N).contiguous()
+    dW = torch.empty(E, K, N, dtype=torch.bfloat16, device="cuda")
+    gg.wgrad(A, dY, offs_d, dW, status=st[1:2])
+    torch.cuda.synchronize()
+    s = st.cpu().numpy()
+    assert np.all(s & gg.DEV_LAUNCHED) and not np.any(s & gg.DEV_ERROR_MASK), s
+    want = torch.tensor([float(m * (e + 1)) for e, m in enumerate(sizes)],
+                        dtype=torch.float32).to(torch.bfloat16).cuda()
+    assert bool((dW[:, 0, :] == want[:, None]).all()), "wgrad: probe row"
+    assert bool((dW[:, 1:, :] == 0).all()), "wgrad: zero rows"
+
+
+@pytest.mark.slow
 def test_gateup_config_full_elementwise():
     """The E=64 Zipf gate-up config (K=2048, N=1536, 4 empty experts, unaligned sizes) in full:
     every element of out, dX (all rows of every group) and dW against the oracle, with NaN
