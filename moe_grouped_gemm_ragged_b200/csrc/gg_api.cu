@@ -235,9 +235,13 @@ bool map_w(CUtensorMap* m, const void* W, int64_t E, int64_t K, int64_t N, uint3
 
 template <Mode MODE, int BN, int STAGES, bool PAIR, bool F32 = false, int ACT = 0>
 gg_status launch(const CUtensorMap& a, const CUtensorMap& b, const gg::Params& p,
-                 int64_t tiles_upper, const DeviceInfo& di, cudaStream_t stream) {
+                 int64_t tiles_upper, const DeviceInfo& di, cudaStream_t stream,
+                 const CUtensorMap* c = nullptr) {
   auto kern = gg::grouped_gemm_kernel<MODE, BN, STAGES, PAIR, F32, ACT>;
-  using L = gg::Layout<BN, STAGES, PAIR, gg::bk_of<MODE>()>;
+  using L = gg::Layout<BN, STAGES, PAIR, gg::bk_of<MODE>(),
+                       gg::staging_bytes<MODE, BN, PAIR, F32, ACT>()>;
+  static_assert(L::bytes(GG_MAX_EXPERTS) <= 227u * 1024u, "shared memory of a CTA exceeded");
+  const CUtensorMap& mc = c != nullptr ? *c : a;  // the output map, where the kernel stores by TMA
   const size_t smem = L::bytes(p.E);
   const int dev = di.dev;
   cudaError_t ce = cudaSuccess;
@@ -303,12 +307,12 @@ gg_status launch(const CUtensorMap& a, const CUtensorMap& b, const gg::Params& p
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  ce = cudaLaunchKernelEx(&cfg, kern, a, b, p);
+  ce = cudaLaunchKernelEx(&cfg, kern, a, b, mc, p);
   if (ce != cudaSuccess && pdl) {
     // a stream or capture that does not take programmatic launches: launch plainly
     (void)cudaGetLastError();
     cfg.numAttrs = na - 1;
-    ce = cudaLaunchKernelEx(&cfg, kern, a, b, p);
+    ce = cudaLaunchKernelEx(&cfg, kern, a, b, mc, p);
   }
   if (ce != cudaSuccess) return cuda_fail("cudaLaunchKernelEx", ce);
   ce = cudaGetLastError();
@@ -358,6 +362,10 @@ constexpr int kPairStages = 6;  // CTA pair: 32 KB per stage and CTA
 constexpr int kWgBK = gg::bk_of<Mode::Wgrad>();  // token rows per wgrad stage
 constexpr int kWgStages = kStages;
 constexpr int kWgPairStages = kPairStages;
+// bf16 wgrad of CTA pairs with 256-column tiles stores dW through 32 KB of shared memory and
+// TMA, which leaves room for five operand stages
+constexpr int kWgPairStagesTma = gg::tma_store_epilogue<Mode::Wgrad, 256, true, false, 0>()
+                                     ? 5 : kWgPairStages;
 // Wide CTA-pair tiles: 256 x 512 with one accumulator (all 512 TMEM columns), 48 KB per
 // stage and CTA. Per flop they move a quarter less operand data into shared memory than
 // 256 x 256 pair tiles and, in wgrad, cover twice as much of dW per wave.
@@ -449,7 +457,13 @@ gg_status wgrad_impl(const void* A, const void* dY, const int32_t* offs, void* d
   if (pair) {
     const int64_t tiles = (int64_t)E * cdiv(K, 2 * gg::BM) * cdiv(N, kBN);
     if (f32) return launch<Mode::Wgrad, kBN, kWgPairStages, true, true>(ma, mb, p, tiles, di, stream);
-    return launch<Mode::Wgrad, kBN, kWgPairStages, true>(ma, mb, p, tiles, di, stream);
+    // dW as [E][K][N] for the tensor stores: boxes of 64 columns x 32 rows of one expert
+    CUtensorMap mc;
+    const uint64_t dims[3] = {(uint64_t)N, (uint64_t)K, (uint64_t)E};
+    const uint64_t str[2] = {(uint64_t)N * 2u, (uint64_t)K * (uint64_t)N * 2u};
+    const uint32_t box[3] = {64u, 32u, 1u};
+    if (!make_map(&mc, dW, 3, dims, str, box)) return GG_ERR_CUDA;
+    return launch<Mode::Wgrad, kBN, kWgPairStagesTma, true>(ma, mb, p, tiles, di, stream, &mc);
   }
   const int64_t tiles = (int64_t)E * cdiv(K, gg::BM) * cdiv(N, kBN);
   if (f32) return launch<Mode::Wgrad, kBN, kWgStages, false, true>(ma, mb, p, tiles, di, stream);

@@ -143,7 +143,22 @@ struct Params {
   int32_t gate_up_concat;
 };
 
-template <int BN, int STAGES, bool PAIR, int BKL = BK>
+// Wgrad of CTA pairs with 256-column tiles and bf16 output stores dW through shared memory
+// and TMA: each epilogue warp stages 32 rows x 64 columns (4 KB, 128-byte swizzle) at a time
+// and issues one tensor store per block (0: predicated stores from registers).
+#ifndef GG_WG_TMA_STORE
+#define GG_WG_TMA_STORE 1
+#endif
+template <Mode MODE, int BN, bool PAIR, bool F32, int ACT>
+__host__ __device__ constexpr bool tma_store_epilogue() {
+  return GG_WG_TMA_STORE && MODE == Mode::Wgrad && PAIR && BN == 256 && !F32 && ACT == 0;
+}
+template <Mode MODE, int BN, bool PAIR, bool F32, int ACT>
+__host__ __device__ constexpr uint32_t staging_bytes() {
+  return tma_store_epilogue<MODE, BN, PAIR, F32, ACT>() ? EPI_WARPS * 4096u : 0u;
+}
+
+template <int BN, int STAGES, bool PAIR, int BKL = BK, uint32_t STG = 0>
 struct Layout {
   static constexpr int B_COLS = PAIR ? BN / 2 : BN;  // columns of B this CTA loads
   static constexpr uint32_t A_BYTES = BM * BKL * 2;
@@ -153,7 +168,8 @@ struct Layout {
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr uint32_t OFF_A = 0;
   static constexpr uint32_t OFF_B = STAGES * A_BYTES;
-  static constexpr uint32_t OFF_BAR = STAGES * STAGE_BYTES;
+  static constexpr uint32_t OFF_STG = STAGES * STAGE_BYTES;  // epilogue staging (STG bytes)
+  static constexpr uint32_t OFF_BAR = OFF_STG + STG;
   // full, empty, landed, fixed (wgrad tail blocks) per stage; tfull x2, tempty x2, fin
   static constexpr uint32_t NUM_BARS = 4 * STAGES + 5;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NUM_BARS * 8;
@@ -402,9 +418,11 @@ __device__ __forceinline__ Tile decode_tile(int32_t t, const Params& p, const Sh
 template <Mode MODE, int BN, int STAGES, bool PAIR, bool F32 = false, int ACT = 0>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap mapA,
-                        const __grid_constant__ CUtensorMap mapB, const Params p) {
+                        const __grid_constant__ CUtensorMap mapB,
+                        const __grid_constant__ CUtensorMap mapC, const Params p) {
   constexpr int BKM = bk_of<MODE>();  // reduction elements per stage
-  using L = Layout<BN, STAGES, PAIR, BKM>;
+  constexpr bool TMA_EPI = tma_store_epilogue<MODE, BN, PAIR, F32, ACT>();
+  using L = Layout<BN, STAGES, PAIR, BKM, staging_bytes<MODE, BN, PAIR, F32, ACT>()>;
   static_assert(BN % 64 == 0 && BN >= 64 && (BN <= 256 || (BN == 512 && PAIR)),
                 "BN must be 64, 128, 192 or 256, or 512 for a CTA pair");
   static_assert(!PAIR || BN % 128 == 0, "a CTA pair splits BN into two multiples of 64");
@@ -470,6 +488,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::fence_mbar_init();
     ptx::prefetch_tmap(&mapA);
     ptx::prefetch_tmap(&mapB);
+    if constexpr (TMA_EPI) ptx::prefetch_tmap(&mapC);
   }
   if (warp == 1) {
     if constexpr (PAIR) {
@@ -1018,6 +1037,47 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
         }
+      } else if constexpr (TMA_EPI) {
+        // dW through shared memory and TMA: the warp's 128 columns in two blocks of 64, each
+        // staged as 32 rows x 128 bytes (16-byte chunk j of row i at chunk j ^ (i % 8), the
+        // 128-byte swizzle of the store's tensor map) and written by one tensor store; the map
+        // covers dW as [E][K][N], so rows past K and columns past N are not written
+        uint8_t* stg = smem + L::OFF_STG + (warp - 2) * 4096u;
+        const uint32_t taddr = tmem_base + ((q * 32u) << 16) + a * BN + (uint32_t)c_off;
+        const int32_t krow = tl.k0 + (int32_t)(rank * BM + q * 32);  // dW row of lane 0
+#pragma unroll 1
+        for (int blk = 0; blk < 2; ++blk) {
+          uint32_t r0[32], r1[32];
+          ptx::tmem_ld_32x32b_x32(taddr + blk * 64, r0);
+          ptx::tmem_ld_32x32b_x32(taddr + blk * 64 + 32, r1);
+          ptx::tmem_ld_wait();
+          uint32_t packed[32];
+#pragma unroll
+          for (int h = 0; h < 16; ++h) {
+            __nv_bfloat162 b0 = __floats2bfloat162_rn(__uint_as_float(r0[2 * h]),
+                                                      __uint_as_float(r0[2 * h + 1]));
+            __nv_bfloat162 b1 = __floats2bfloat162_rn(__uint_as_float(r1[2 * h]),
+                                                      __uint_as_float(r1[2 * h + 1]));
+            packed[h] = *reinterpret_cast<uint32_t*>(&b0);
+            packed[16 + h] = *reinterpret_cast<uint32_t*>(&b1);
+          }
+          if (lane == 0) ptx::bulk_wait_read_all();  // the last store has read the buffer
+          __syncwarp();
+          uint8_t* row = stg + lane * 128u;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(row + ((j ^ (int)(lane & 7u)) * 16)) =
+                make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          // a box wholly past K or N (the last tiles of a K or N that is not a multiple of
+          // the tile) is not stored at all; a box that only reaches past them is clipped
+          const int32_t xcol = tl.n0 + c_off + blk * 64;
+          if (lane == 0 && xcol < p.out_cols && krow < p.wg_K) {
+            ptx::tma_store_3d(&mapC, stg, xcol, krow, tl.e);
+            ptx::bulk_commit_group();
+          }
+        }
       } else {
       const uint32_t taddr = tmem_base + ((q * 32u) << 16) + a * BN + (uint32_t)c_off;
       // 32 columns per load; the next load is in flight while this chunk is stored
@@ -1129,6 +1189,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       ++acc_iter;
+    }
+    if constexpr (TMA_EPI) {
+      // every tensor store of this warp has written dW before the CTA can exit
+      if (lane == 0) ptx::bulk_wait_all();
+      __syncwarp();
     }
   } else if constexpr (MODE == Mode::Wgrad) {
     // ------------------------------------------------------------ wgrad tail fix-up
