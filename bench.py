@@ -537,15 +537,41 @@ def masked_timings(gg, m, dev, peaks, copies: int = 16, rounds: int = 12):
         del g
         return a.elapsed_time(b) * 1e3 / len(seq)
 
+    def single_after_us(dirty: bool, reps: int = 20):
+        """One eager call (event to event) right after a 256 MB pass that leaves L2 full of
+        clean lines (a read) or of dirty ones (a write, as the output stores of a preceding
+        GEMM do): with dirty lines every line the call brings in first writes one back."""
+        buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        acc = torch.empty((), dtype=torch.int64, device=dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ts = []
+        for r in range(reps):
+            if dirty:
+                buf.fill_(r & 0xFF)
+            else:
+                torch.sum(buf.view(torch.int64), out=acc)
+            i = r % copies
+            a.record()
+            gg.masked_forward(As[i], Ws[i], mm, outs[i])
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b) * 1e3)
+        del buf
+        return float(np.median(ts))
+
     gg.masked_forward(As[0], Ws[0], mm, outs[0])
     torch.cuda.synchronize()
     hot = float(np.median([per_call_us([0] * 200) for _ in range(3)]))
     cold = float(np.median([per_call_us(list(range(copies)) * rounds) for _ in range(3)]))
+    after_clean = single_after_us(False)
+    after_dirty = single_after_us(True)
     nbytes = masked_bytes(m)
     return {"algorithmic_bytes": nbytes, "hot_graph_us": hot, "cold_graph_us": cold,
             "cold_gbs": nbytes / (cold * 1e-6) / 1e9,
             "cold_frac_of_hbm": nbytes / (cold * 1e-6) / 1e9 / peaks["hbm_gbs"],
             "hot_gbs": nbytes / (hot * 1e-6) / 1e9,
+            "single_after_clean_l2_us": after_clean,
+            "single_after_dirty_l2_us": after_dirty,
             "kernel": "masked_forward_kernel (weight columns as the MMA's M)"}
 
 
