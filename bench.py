@@ -549,7 +549,7 @@ def masked_timings(gg, m, dev, peaks, copies: int = 16, rounds: int = 12):
             if dirty:
                 buf.fill_(r & 0xFF)
             else:
-                torch.sum(buf.view(torch.int64), out=acc)
+                torch.sum(buf.view(torch.int64), dim=0, out=acc)
             i = r % copies
             a.record()
             gg.masked_forward(As[i], Ws[i], mm, outs[i])
