@@ -36,16 +36,16 @@ UNIT = "TFLOP/s"
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant kernel,
 # keyed by pass and workload, valid only for the kernel sources whose hash is recorded with
-# them (a changed kernel reports null until it is captured again). Each figure comes from a
-# capture of ONE launch of ONE kernel (-k <kernel> -c 1) with only these counters, which ncu
-# collects in a single pass; a launch list over many kernels collects gpu__time_duration.sum
-# alone.
+# them (a changed kernel reports null until it is captured again). The figures come from one
+# capture of the second launch of each pass (-k regex:grouped_gemm -s 3 -c 3) with only these
+# counters, which ncu collects in a single pass (nothing saved or restored); a launch list over
+# many kernels collects gpu__time_duration.sum alone.
 NCU_TRAFFIC = {
-    ("forward", "large"): 11.103e9,
-    ("dgrad", "large"): 12.583e9,
-    ("wgrad", "large"): 19.867e9,
+    ("forward", "large"): 14.383e9,
+    ("dgrad", "large"): 14.032e9,
+    ("wgrad", "large"): 20.106e9,
 }
-NCU_TRAFFIC_SRC_HASH = "5794e31d918ee2ec"
+NCU_TRAFFIC_SRC_HASH = "dd8c5dac2de7eced"
 
 
 GEMM_SOURCES = ("gg_kernel.cuh", "ptx.cuh", "gg_api.cu", "gg_masked.cuh")  # kernels + launch
@@ -187,6 +187,16 @@ def make_clock_sampler(device_index: int):
         return NvmlClockSampler(device_index)
     except Exception:
         return ClockSampler(device_index)
+
+
+def clocked(fn, device_index: int):
+    """Runs fn() with the SM clock sampled meanwhile: (fn's result, median SM MHz or None).
+    Kernels that are latency-bound (the masked forward, the small configs) scale with it."""
+    sampler = make_clock_sampler(device_index)
+    sampler.start()
+    res = fn()
+    c = sampler.stop()
+    return res, (c or {}).get("sm_mhz")
 
 
 def reduce_max(value: float, device) -> float:
@@ -501,9 +511,10 @@ def run_config_extras(gg, dev, stream, peaks, reps: int):
                  "group_sizes": f"min {int(r.sizes.min())} max {int(r.sizes.max())}, "
                                 f"{int((r.sizes == 0).sum())} empty"}
         for pas, fn in fns.items():
-            ms = _median_call_ms(fn, stream, reps)
+            ms, mhz = clocked(lambda: _median_call_ms(fn, stream, reps), dev.index)
             tf = r.flops / (ms * 1e-3) / 1e12
-            entry[pas] = {"ms": ms, "tflops": tf, "frac_of_burst": tf / peaks["bf16_tflops"]}
+            entry[pas] = {"ms": ms, "tflops": tf, "frac_of_burst": tf / peaks["bf16_tflops"],
+                          "sm_mhz": mhz}
         res[name] = entry
         del r, offs, out, dX, dW, fns
         torch.cuda.empty_cache()
@@ -561,8 +572,10 @@ def masked_timings(gg, m, dev, peaks, copies: int = 16, rounds: int = 12):
 
     gg.masked_forward(As[0], Ws[0], mm, outs[0])
     torch.cuda.synchronize()
-    hot = float(np.median([per_call_us([0] * 200) for _ in range(3)]))
-    cold = float(np.median([per_call_us(list(range(copies)) * rounds) for _ in range(3)]))
+    hot, hot_mhz = clocked(lambda: float(np.median([per_call_us([0] * 200)
+                                                    for _ in range(3)])), dev.index)
+    cold, cold_mhz = clocked(lambda: float(np.median([per_call_us(list(range(copies)) * rounds)
+                                                      for _ in range(3)])), dev.index)
     after_clean = single_after_us(False)
     after_dirty = single_after_us(True)
     nbytes = masked_bytes(m)
@@ -570,6 +583,7 @@ def masked_timings(gg, m, dev, peaks, copies: int = 16, rounds: int = 12):
             "cold_gbs": nbytes / (cold * 1e-6) / 1e9,
             "cold_frac_of_hbm": nbytes / (cold * 1e-6) / 1e9 / peaks["hbm_gbs"],
             "hot_gbs": nbytes / (hot * 1e-6) / 1e9,
+            "hot_sm_mhz": hot_mhz, "cold_sm_mhz": cold_mhz,
             "single_after_clean_l2_us": after_clean,
             "single_after_dirty_l2_us": after_dirty,
             "kernel": "masked_forward_kernel (weight columns as the MMA's M)"}
