@@ -381,15 +381,17 @@ bool use_pair(int64_t rows, int32_t E) {
   return rows >= 512 * (int64_t)E;
 }
 
-// Forward and dgrad on 256 x 512 CTA-pair tiles where CTA pairs are used and the reduction
-// is long: the tile's epilogue no longer overlaps the next mainloop, which a long reduction
-// amortises (large shape, reduction 6144 / 4096: forward 1279 vs 1205 TFLOP/s, dgrad 1219 vs
-// 1188 in alternating runs; down-proj forward, reduction 2048: 1158 vs 1221).
+// Forward and dgrad on 256 x 512 CTA-pair tiles wherever CTA pairs are used: per flop they
+// bring a quarter less operand data from L2 into shared memory, and the operand supply is
+// what bounds the 256 x 256 tiles (alternating runs at 1965 MHz, wide vs 256 x 256: gate-up
+// forward 994 vs 976 TFLOP/s and dgrad 978 vs 944, down-proj forward 1323 vs 1274 and dgrad
+// 1405 vs 1313; large shape forward 1279 vs 1205, dgrad 1219 vs 1188).
 bool use_wide(int64_t rows, int32_t E, int64_t red_len) {
+  (void)red_len;
   const int v = g_force_variant.load();
   if (v == 1 || v == 2) return false;
   if (v == 3) return true;
-  return rows >= 512 * (int64_t)E && red_len >= 4096;
+  return use_pair(rows, E);
 }
 
 // Wgrad launch shape: 0 single CTAs, 1 CTA pairs, 2 wide CTA pairs. A wgrad tile is as long
