@@ -45,7 +45,8 @@ def _buffers(rows, E):
     s = workloads.sentinel_like
     return {"y1": s((rows, D)).cuda(), "y2": s((rows, D)).cuda(), "g": s((rows, D)).cuda(),
             "dW": s((E, D, D)).cuda(), "offs2": torch.zeros(E, dtype=torch.int32, device="cuda"),
-            "y3": s((rows, D)).cuda(), "mout": s((E, MMAX, D)).cuda()}
+            "y3": s((rows, D)).cuda(), "y4": s((rows, D)).cuda(),
+            "mout": s((E, MMAX, D)).cuda()}
 
 
 def _chain(r, W2, offs, offs_alt, masked_m, b, sync: bool):
@@ -55,6 +56,7 @@ def _chain(r, W2, offs, offs_alt, masked_m, b, sync: bool):
     gg.forward(b["y1"], W2, offs, b["y2"]); step()          # reads y1
     gg.dgrad(b["y2"], W2, offs, b["g"]); step()             # reads y2
     gg.wgrad(b["y1"], b["g"], offs, b["dW"]); step()        # reads g, written just before
+    gg.forward(b["g"], b["dW"], offs, b["y4"]); step()      # reads dW (all of a split wgrad)
     b["offs2"].copy_(offs_alt); step()                      # offsets from a torch kernel
     gg.forward(b["g"], r.W, b["offs2"], b["y3"]); step()    # reads g and the new offsets
     mA = b["y3"][:E * MMAX].view(E, MMAX, D)
