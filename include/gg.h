@@ -305,7 +305,8 @@ GG_API int gg_testing_skip_first_load(int enable);
 
 /* Test hook: choose the launch shape of gg_forward, gg_dgrad and gg_wgrad for later calls:
    0 = automatic (forward/dgrad: CTA pairs with 256 x 512 tiles when rows_alloc >= 512*E,
-   else single CTAs; wgrad: by the average group length), 1 = single CTAs (128 x 256 tiles),
+   with the SiLU-and-mul epilogue only when K >= 4096 (else 256 x 256), else single CTAs;
+   wgrad: by the average group length), 1 = single CTAs (128 x 256 tiles),
    2 = CTA pairs (256 x 256 tiles on two SMs), 3 = CTA pairs with 256 x 512 tiles.
    Results are the same up to rounding order.
    Returns the previous setting. */

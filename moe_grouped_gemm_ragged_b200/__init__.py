@@ -120,7 +120,8 @@ def testing_skip_first_load(enable: bool) -> bool:
 
 def testing_force_variant(variant: int) -> int:
     """Test hook: 0 automatic, 1 single-CTA tiles, 2 CTA-pair tiles, 3 wide CTA pairs
-    (256 x 512 tiles, the automatic forward/dgrad shape of CTA pairs), each for every pass."""
+    (256 x 512 tiles, the automatic forward/dgrad shape of CTA pairs, and of the SiLU-and-mul
+    forward when K >= 4096), each for every pass."""
     return int(lib().gg_testing_force_variant(int(variant)))
 
 

@@ -385,13 +385,16 @@ bool use_pair(int64_t rows, int32_t E) {
 // bring a quarter less operand data from L2 into shared memory, and the operand supply is
 // what bounds the 256 x 256 tiles (alternating runs at 1965 MHz, wide vs 256 x 256: gate-up
 // forward 994 vs 976 TFLOP/s and dgrad 978 vs 944, down-proj forward 1323 vs 1274 and dgrad
-// 1405 vs 1313; large shape forward 1279 vs 1205, dgrad 1219 vs 1188).
-bool use_wide(int64_t rows, int32_t E, int64_t red_len) {
-  (void)red_len;
+// 1405 vs 1313; large shape forward 1279 vs 1205, dgrad 1219 vs 1188). The SiLU-and-mul
+// epilogue of a wide tile releases its accumulator only after its stores, which a short
+// reduction does not hide: with it, wide tiles only from a reduction of 4096 on (SiLU
+// forward, wide vs 256 x 256: large slice 1503 vs 1440; gate-up 917 vs 1003, down-proj 1199
+// vs 1302).
+bool use_wide(int64_t rows, int32_t E, int64_t red_len, bool silu = false) {
   const int v = g_force_variant.load();
   if (v == 1 || v == 2) return false;
   if (v == 3) return true;
-  return use_pair(rows, E);
+  return use_pair(rows, E) && (!silu || red_len >= 4096);
 }
 
 // Wgrad launch shape: 0 single CTAs, 1 CTA pairs, 2 wide CTA pairs. A wgrad tile is as long
@@ -510,7 +513,7 @@ gg_status forward_impl(const void* A, const void* W, const int32_t* offs, void* 
   // [gate | up] weights are loaded as 128-column gate and up blocks
   const bool concat = (flags & GG_FLAG_GATE_UP_CONCAT) != 0;
   const bool pair = use_pair(rows_alloc, E);
-  const bool wide = pair && use_wide(rows_alloc, E, K);
+  const bool wide = pair && use_wide(rows_alloc, E, K, silu);
   const bool chunked = (N % 64) == 0;
   const uint32_t bcols = wide ? kWideBN / 2 : pair ? kBN / 2 : kBN;
   const uint32_t bbox = concat ? 128u : bcols;  // columns of W per box
