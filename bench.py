@@ -41,11 +41,11 @@ UNIT = "TFLOP/s"
 # counters, which ncu collects in a single pass (nothing saved or restored); a launch list over
 # many kernels collects gpu__time_duration.sum alone.
 NCU_TRAFFIC = {
-    ("forward", "large"): 16.895e9,
-    ("dgrad", "large"): 14.743e9,
-    ("wgrad", "large"): 26.316e9,
+    ("forward", "large"): 10.760e9,
+    ("dgrad", "large"): 12.944e9,
+    ("wgrad", "large"): 14.378e9,
 }
-NCU_TRAFFIC_SRC_HASH = "3db59a5c9134e27b"
+NCU_TRAFFIC_SRC_HASH = "a0da491e0ea04d57"
 
 
 GEMM_SOURCES = ("gg_kernel.cuh", "ptx.cuh", "gg_api.cu", "gg_masked.cuh")  # kernels + launch
