@@ -29,8 +29,9 @@ constexpr int CHUNK = THREADS;        // assignments per block
 constexpr int32_t DEV_BAD_ROUTE = 0x8;
 static_assert(DEV_BAD_ROUTE == GG_DEV_BAD_ROUTE, "status bit mismatch");
 
-// Histogram of the block's chunk: counts[b * E + e] (ids < 0 are dropped silently, ids >= E
-// are dropped and flagged).
+// Histogram of the block's chunk: counts[e * nblk + b] for block b of nblk (ids < 0 are dropped
+// silently, ids >= E are dropped and flagged). Expert-major, so that the scan reads the
+// counts of one expert with consecutive lanes.
 __global__ void __launch_bounds__(THREADS) count_kernel(const int32_t* __restrict__ ids,
                                                         int64_t n, int32_t E,
                                                         int32_t* __restrict__ counts,
@@ -46,71 +47,83 @@ __global__ void __launch_bounds__(THREADS) count_kernel(const int32_t* __restric
     bad = e >= E;
   }
   bad = __syncthreads_or(bad);
-  for (int e = threadIdx.x; e < E; e += THREADS) counts[(int64_t)blockIdx.x * E + e] = hist[e];
+  for (int e = threadIdx.x; e < E; e += THREADS)
+    counts[(int64_t)e * gridDim.x + blockIdx.x] = hist[e];
   if (bad && threadIdx.x == 0 && status != nullptr) atomicOr(status, DEV_BAD_ROUTE);
 }
 
-// One block: offs[e] = cumulative end of expert e; counts[b][e] becomes the first packed row
-// of block b's assignments to expert e. G threads share an expert (G a power of two, at most
-// 32 and at most 1024 / E), each owning a contiguous run of blocks, so that the serial walk
-// over the histograms is nblk / G long instead of nblk.
-__global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ counts, int32_t nblk,
-                                                    int32_t E, int32_t* __restrict__ offs) {
-  __shared__ int32_t tot[GG_MAX_EXPERTS];  // per expert: total, then exclusive start
-  __shared__ int32_t warp_sum[32];
-  int lg = 5;
-  while (lg > 0 && (E << lg) > 1024) --lg;
-  const int G = 1 << lg;
-  const int e = threadIdx.x >> lg, s = threadIdx.x & (G - 1);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const bool own = e < E;
-  const int32_t span = (nblk + G - 1) / G;
-  const int32_t b0 = min(s * span, nblk), b1 = min(b0 + span, nblk);
-  int32_t seg = 0;
-  if (own) {
-#pragma unroll 8
-    for (int32_t b = b0; b < b1; ++b) seg += counts[(int64_t)b * E + e];
-  }
-  // inclusive scan of the run sums over the G threads of the expert (a G-aligned lane group)
-  int32_t run_incl = seg;
-  for (int d = 1; d < G; d <<= 1) {
-    const int32_t o = __shfl_up_sync(0xffffffffu, run_incl, d);
-    if (s >= d) run_incl += o;
-  }
-  const int32_t total = __shfl_sync(0xffffffffu, run_incl, lane | (G - 1));
-  if (own && s == 0) tot[e] = total;
-  __syncthreads();
-  // block-wide exclusive scan of the totals over experts (thread x takes expert x)
-  const int32_t tx = (int)threadIdx.x < E ? tot[threadIdx.x] : 0;
-  int32_t v = tx;
+// One block: offs[e] = cumulative end of expert e; counts[e][b] becomes the first packed row
+// of block b's assignments to expert e. Each expert's blocks are cut into P segments (P a
+// power of two, 32 / E rounded down for fewer than 32 experts, else 1), one warp per segment
+// at a time: the warp sums its segment with consecutive lanes on consecutive blocks, one
+// exclusive scan runs over the E * P segment sums in (expert, segment) order, and each warp
+// then turns its segment's counts into starts with a running warp-wide scan.
+__device__ __forceinline__ int32_t warp_incl_scan(int32_t v, int lane) {
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
     const int32_t o = __shfl_up_sync(0xffffffffu, v, d);
     if (lane >= d) v += o;
   }
-  if (lane == 31) warp_sum[warp] = v;
-  __syncthreads();
-  if (warp == 0) {
-    int32_t w = warp_sum[lane];
+  return v;
+}
+
+__global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ counts, int32_t nblk,
+                                                    int32_t E, int32_t* __restrict__ offs) {
+  constexpr int U = 8;                        // loads in flight per lane
+  __shared__ int32_t seg[GG_MAX_EXPERTS];     // per segment: sum, then exclusive start
+  __shared__ int32_t warp_sum[32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int P = 1;
+  while (P * 2 * E <= 32) P *= 2;
+  const int32_t S = E * P;                    // at most GG_MAX_EXPERTS segments
+  const int32_t span = (nblk + P - 1) / P;
+  // segment sg = e * P + p covers blocks [p * span, min((p + 1) * span, nblk)) of expert e
+  for (int32_t sg = warp; sg < S; sg += 32) {
+    const int32_t e = sg / P, p = sg % P;
+    const int32_t b0 = min(p * span, nblk), b1 = min(b0 + span, nblk);
+    const int32_t* row = counts + (int64_t)e * nblk;
+    int32_t sum = 0;
+    for (int32_t b = b0 + lane; b < b1; b += 32 * U) {
+      int32_t c[U];
 #pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-      const int32_t o = __shfl_up_sync(0xffffffffu, w, d);
-      if (lane >= d) w += o;
+      for (int u = 0; u < U; ++u) c[u] = b + 32 * u < b1 ? row[b + 32 * u] : 0;
+#pragma unroll
+      for (int u = 0; u < U; ++u) sum += c[u];
     }
-    warp_sum[lane] = w;
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, d);
+    if (lane == 0) seg[sg] = sum;
   }
   __syncthreads();
-  if ((int)threadIdx.x < E) tot[threadIdx.x] = v + (warp > 0 ? warp_sum[warp - 1] : 0) - tx;
+  // block-wide exclusive scan of the segment sums (thread x takes segment x); the end of an
+  // expert's last segment is its cumulative end offset
+  const int32_t tx = (int)threadIdx.x < S ? seg[threadIdx.x] : 0;
+  const int32_t v = warp_incl_scan(tx, lane);
+  if (lane == 31) warp_sum[warp] = v;
   __syncthreads();
-  if (own) {
-    const int32_t start = tot[e];
-    if (s == 0) offs[e] = start + total;
-    int32_t run = start + run_incl - seg;
-#pragma unroll 8
-    for (int32_t b = b0; b < b1; ++b) {
-      const int32_t c = counts[(int64_t)b * E + e];
-      counts[(int64_t)b * E + e] = run;
-      run += c;
+  if (warp == 0) warp_sum[lane] = warp_incl_scan(warp_sum[lane], lane);
+  __syncthreads();
+  if ((int)threadIdx.x < S) {
+    const int32_t incl = v + (warp > 0 ? warp_sum[warp - 1] : 0);
+    seg[threadIdx.x] = incl - tx;
+    if ((int)threadIdx.x % P == P - 1) offs[threadIdx.x / P] = incl;
+  }
+  __syncthreads();
+  for (int32_t sg = warp; sg < S; sg += 32) {
+    const int32_t e = sg / P, p = sg % P;
+    const int32_t b0 = min(p * span, nblk), b1 = min(b0 + span, nblk);
+    int32_t* row = counts + (int64_t)e * nblk;
+    int32_t carry = seg[sg];
+    for (int32_t b = b0 + lane; b - lane < b1; b += 32 * U) {
+      int32_t c[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) c[u] = b + 32 * u < b1 ? row[b + 32 * u] : 0;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int32_t incl = warp_incl_scan(c[u], lane);
+        if (b + 32 * u < b1) row[b + 32 * u] = carry + incl - c[u];
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+      }
     }
   }
 }
@@ -134,7 +147,7 @@ __global__ void __launch_bounds__(THREADS) scatter_kernel(
   __syncthreads();
   // exclusive scan over warps per expert, starting at the block's base
   for (int x = threadIdx.x; x < E; x += THREADS) {
-    int32_t run = bases[(int64_t)blockIdx.x * E + x];
+    int32_t run = bases[(int64_t)x * gridDim.x + blockIdx.x];
     for (int w = 0; w < WARPS; ++w) {
       const int32_t c = whist[w * E + x];
       whist[w * E + x] = run;
