@@ -28,8 +28,11 @@ def _route(ids, X, E):
 
 @pytest.mark.parametrize("T,k,E,K,dropped", [(37, 3, 6, 16, 4), (4096, 8, 64, 2048, 0),
                                              (1000, 4, 1024, 64, 100), (5, 1, 1, 8, 0),
-                                             (300, 2, 33, 136, 599)])
+                                             (300, 2, 33, 136, 599), (4096, 4, 8, 64, 0),
+                                             (20000, 2, 3, 16, 50)])
 def test_route_bit_exact(T, k, E, K, dropped):
+    """Stable routing equal to the oracle's; the last two cases split each expert's 64 and
+    157 per-block histograms into 4 and 8 scan segments (the last one partial)."""
     ids, X = workloads.make_routing(T, k, E, K, seed=T + E, dropped=min(dropped, T * k))
     Ap, row_of, offs, st = _route(ids, X, E)
     roffs, rrow, rA, bad = oracle.route(ids, X, E)
