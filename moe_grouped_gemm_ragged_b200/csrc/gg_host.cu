@@ -2,7 +2,11 @@
 // streamed through the GPU by expert chunks: while chunk c computes on the caller's stream,
 // the operands of chunk c+1 travel host -> device on one copy stream and the results of
 // chunk c-1 travel device -> host on another (the host link is full duplex), so a pass costs
-// about the larger of the two transfers instead of their sum plus the GEMMs.
+// about the larger of the two transfers instead of their sum plus the GEMMs. Each pass waits
+// only for its own operands and each result leaves as soon as its pass is done: W and A
+// travel first and the forward starts while dY is still on its way, and the forward's
+// output goes back while dgrad and wgrad run, which shortens the start and the end of the
+// pipeline.
 #include <cstdint>
 #include <mutex>
 
@@ -23,7 +27,9 @@ struct DeviceCtx {
   bool ready = false;
   cudaStream_t h2d = nullptr, d2h = nullptr;
   cudaEvent_t start = nullptr, done = nullptr;
-  cudaEvent_t loaded[kMaxChunks] = {}, computed[kMaxChunks] = {};
+  // per chunk: W and A loaded, dY loaded; forward, dgrad and wgrad done
+  cudaEvent_t loaded_aw[kMaxChunks] = {}, loaded[kMaxChunks] = {};
+  cudaEvent_t fwd_done[kMaxChunks] = {}, dgrad_done[kMaxChunks] = {}, computed[kMaxChunks] = {};
 };
 std::mutex g_mu;
 DeviceCtx g_ctx[kMaxDevices];
@@ -41,7 +47,10 @@ gg_status device_ctx(DeviceCtx** out) {
         cudaEventCreateWithFlags(&c.done, ef) != cudaSuccess)
       return GG_ERR_CUDA;
     for (int i = 0; i < kMaxChunks; ++i)
-      if (cudaEventCreateWithFlags(&c.loaded[i], ef) != cudaSuccess ||
+      if (cudaEventCreateWithFlags(&c.loaded_aw[i], ef) != cudaSuccess ||
+          cudaEventCreateWithFlags(&c.loaded[i], ef) != cudaSuccess ||
+          cudaEventCreateWithFlags(&c.fwd_done[i], ef) != cudaSuccess ||
+          cudaEventCreateWithFlags(&c.dgrad_done[i], ef) != cudaSuccess ||
           cudaEventCreateWithFlags(&c.computed[i], ef) != cudaSuccess)
         return GG_ERR_CUDA;
     c.ready = true;
@@ -147,33 +156,47 @@ gg_status gg_layer_step_host(const void* A_h, const void* W_h, const void* dY_h,
     const int32_t e0 = ch.e0[c], ne = ch.e0[c + 1] - ch.e0[c];
     const size_t a_off = (size_t)r0 * (size_t)K * eb, y_off = (size_t)r0 * (size_t)N * eb;
     const size_t w_off = (size_t)e0 * w_bytes;
-    if (!ok(cudaMemcpyAsync(at(A_d, a_off), at(A_h, a_off), (size_t)nr * K * eb,
+    // W and A (the forward's operands), then dY
+    if (!ok(cudaMemcpyAsync(at(W_d, w_off), at(W_h, w_off), (size_t)ne * w_bytes,
                             cudaMemcpyHostToDevice, cx->h2d)) ||
+        !ok(cudaMemcpyAsync(at(A_d, a_off), at(A_h, a_off), (size_t)nr * K * eb,
+                            cudaMemcpyHostToDevice, cx->h2d)) ||
+        !ok(cudaEventRecord(cx->loaded_aw[c], cx->h2d)) ||
         !ok(cudaMemcpyAsync(at(dY_d, y_off), at(dY_h, y_off), (size_t)nr * N * eb,
                             cudaMemcpyHostToDevice, cx->h2d)) ||
-        !ok(cudaMemcpyAsync(at(W_d, w_off), at(W_h, w_off), (size_t)ne * w_bytes,
-                            cudaMemcpyHostToDevice, cx->h2d)) ||
         !ok(cudaEventRecord(cx->loaded[c], cx->h2d)) ||
-        !ok(cudaStreamWaitEvent(stream, cx->loaded[c], 0))) {
+        !ok(cudaStreamWaitEvent(stream, cx->loaded_aw[c], 0))) {
       s = GG_ERR_CUDA;
       break;
     }
     const int32_t* offs_c = offs_d + e0;
     s = gg_forward(at(A_d, a_off), at(W_d, w_off), offs_c, at(out_d, y_off), nr, K, N, ne,
                    dev_status, stream);
-    if (s == GG_OK)
-      s = gg_dgrad(at(dY_d, y_off), at(W_d, w_off), offs_c, at(dX_d, a_off), nr, K, N, ne,
-                   dev_status, stream);
-    if (s == GG_OK)
-      s = gg_wgrad(at(A_d, a_off), at(dY_d, y_off), offs_c, at(dW_d, w_off), nr, K, N, ne,
-                   dev_status, stream);
+    if (s != GG_OK) break;
+    // the forward's output leaves while dY arrives and the backward passes run
+    if (!ok(cudaEventRecord(cx->fwd_done[c], stream)) ||
+        !ok(cudaStreamWaitEvent(cx->d2h, cx->fwd_done[c], 0)) ||
+        !ok(cudaMemcpyAsync(at(out_h, y_off), at(out_d, y_off), (size_t)nr * N * eb,
+                            cudaMemcpyDeviceToHost, cx->d2h)) ||
+        !ok(cudaStreamWaitEvent(stream, cx->loaded[c], 0))) {
+      s = GG_ERR_CUDA;
+      break;
+    }
+    s = gg_dgrad(at(dY_d, y_off), at(W_d, w_off), offs_c, at(dX_d, a_off), nr, K, N, ne,
+                 dev_status, stream);
+    if (s != GG_OK) break;
+    if (!ok(cudaEventRecord(cx->dgrad_done[c], stream)) ||
+        !ok(cudaStreamWaitEvent(cx->d2h, cx->dgrad_done[c], 0)) ||
+        !ok(cudaMemcpyAsync(at(dX_h, a_off), at(dX_d, a_off), (size_t)nr * K * eb,
+                            cudaMemcpyDeviceToHost, cx->d2h))) {
+      s = GG_ERR_CUDA;
+      break;
+    }
+    s = gg_wgrad(at(A_d, a_off), at(dY_d, y_off), offs_c, at(dW_d, w_off), nr, K, N, ne,
+                 dev_status, stream);
     if (s != GG_OK) break;
     if (!ok(cudaEventRecord(cx->computed[c], stream)) ||
         !ok(cudaStreamWaitEvent(cx->d2h, cx->computed[c], 0)) ||
-        !ok(cudaMemcpyAsync(at(out_h, y_off), at(out_d, y_off), (size_t)nr * N * eb,
-                            cudaMemcpyDeviceToHost, cx->d2h)) ||
-        !ok(cudaMemcpyAsync(at(dX_h, a_off), at(dX_d, a_off), (size_t)nr * K * eb,
-                            cudaMemcpyDeviceToHost, cx->d2h)) ||
         !ok(cudaMemcpyAsync(at(dW_h, w_off), at(dW_d, w_off), (size_t)ne * w_bytes,
                             cudaMemcpyDeviceToHost, cx->d2h)))
       s = GG_ERR_CUDA;
